@@ -1,0 +1,472 @@
+"""Benchmark of the DiT joint-attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload flux_2048] [--impl ours|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input of the chosen
+workload (default: FLUX-2048-like joint attention, B=1 H=24 S=16896 D=128, bf16):
+    1. dit_attn_fwd         full attention forward (out bf16 + lse)
+    2. dit_attn_fwd_chunk   x n_chunks: the same queries against n equal KV chunks (fp32 partials)
+    3. dit_attn_merge       exact LSE merge of the n partials (bf16 out + lse)
+For the video workload the FP8 variant adds dit_quant_fp8 of Q, K, V and an E4M3 forward.
+
+Metric: TFLOP/s counted as 4*B*H*S^2*D per attention pass (the full pass and the chunked
+pass each count once), whole job, max over ranks.  Inputs (Q, K, V) are resident in HBM and
+larger than the 126 MB L2, so no L2 flush is needed between steps.  Multi-GPU (torchrun):
+every rank runs its own replica batch (independent problems; no data-path collective),
+scaling "weak".
+
+--impl reference times the fp64 CPU oracle (the only other implementation of this path) on
+the host cores, on a bounded sample of the same workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, chunk_bounds, make_qkv  # noqa: E402
+
+METRIC = "DiT attention TFLOP/s (4·B·H·S²·D) and % of B200 dense BF16/FP8 peak, 1 GPU"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_bf16_flux2048.txt")
+KERNEL_SRC = os.path.join(ROOT, "long_sequence_attention_b200", "csrc", "attn_fwd.cuh")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- helpers
+def rank_info():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_hash() -> str:
+    with open(KERNEL_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the full-forward kernel from the committed ncu summary, or
+    None when there is none or the kernel source changed since it was captured."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    vals = {}
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if ":" in line:
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != kernel_hash():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples (every 200 ms) during the timed region."""
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev),
+                 "--query-gpu=clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+                bits = int(parts[3], 16) if parts[3].startswith("0x") else int(parts[3])
+            except ValueError:
+                continue
+            for b, name in REASON_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- our arm
+class Step:
+    """Device buffers and the launch sequence of one step of the hot path."""
+
+    def __init__(self, lsa, w, data, dev, fp8: bool):
+        import torch
+        self.lsa, self.w, self.fp8 = lsa, w, fp8
+        B, H, S, D = w.B, w.H, w.S, w.D
+        to_dev = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+        self.q, self.k, self.v = (to_dev(data[n + "_bits"]) for n in "qkv")
+        self.out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+        self.bounds = chunk_bounds(S, w.n_chunks) if w.n_chunks > 1 else []
+        self.parts = [(torch.empty((B, H, S, D), dtype=torch.float32, device=dev),
+                       torch.empty((B, H, S), dtype=torch.float32, device=dev)) for _ in self.bounds]
+        self.mout = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev)
+        self.mlse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+        if fp8:
+            n = B * H * S * D
+            self.codes = [torch.empty((B, H, S, D), dtype=torch.uint8, device=dev) for _ in range(3)]
+            self.descale = torch.empty((3,), dtype=torch.float32, device=dev)
+            self.ws_bytes = lsa.dit_quant_fp8_workspace_bytes(n)
+            self.ws = torch.empty((self.ws_bytes // 4,), dtype=torch.float32, device=dev)
+            self.out8 = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev)
+            self.lse8 = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+
+    @property
+    def launches(self) -> int:
+        n = 1
+        if self.bounds:
+            n += len(self.bounds) + 1
+        if self.fp8:
+            n += 3 * 2 + 1
+        return n
+
+    @property
+    def flops(self) -> float:
+        f = self.w.flops * (1 + (1 if self.bounds else 0))
+        if self.fp8:
+            f += self.w.flops
+        return f
+
+    def run(self, stream, ev=None):
+        lsa, w = self.lsa, self.w
+        B, H, S, D = w.B, w.H, w.S, w.D
+        if ev is not None:
+            ev[0].record(stream)
+        lsa.dit_attn_fwd(self.q, self.k, self.v, self.out, self.lse, B, H, S, D, w.scale, lsa.DIT_BF16, None, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        for (a, b), (po, pl) in zip(self.bounds, self.parts):
+            lsa.dit_attn_fwd_chunk(self.q, self.k, self.v, po, pl, B, H, S, S, D, a, b, w.scale, lsa.DIT_BF16,
+                                   lsa.DIT_FP32, None, stream)
+        if self.bounds:
+            if ev is not None:
+                ev[2].record(stream)
+            lsa.dit_attn_merge([p[0] for p in self.parts], [p[1] for p in self.parts], self.mout, self.mlse,
+                               B, H, S, D, lsa.DIT_FP32, lsa.DIT_BF16, stream)
+            if ev is not None:
+                ev[3].record(stream)
+        if self.fp8:
+            n = B * H * S * D
+            for i, x in enumerate((self.q, self.k, self.v)):
+                lsa.dit_quant_fp8(x, self.codes[i], self.descale[i:i + 1], n, self.ws, self.ws_bytes, stream)
+            if ev is not None:
+                ev[4].record(stream)
+            lsa.dit_attn_fwd(self.codes[0], self.codes[1], self.codes[2], self.out8, self.lse8, B, H, S, D,
+                             w.scale, lsa.DIT_FP8_E4M3, self.descale, stream)
+            if ev is not None:
+                ev[5].record(stream)
+
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+    import long_sequence_attention_b200 as lsa
+
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    w = WORKLOADS[args.workload]
+    fp8 = args.workload == "video"
+    data = make_qkv(w, seed_offset=rank * 10)          # each rank: its own replica batch
+    stream = torch.cuda.Stream(device=dev)
+    step = Step(lsa, w, data, dev, fp8)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            step.run(stream)
+    stream.synchronize()
+    if lsa.dit_device_status(clear=True) != 0:
+        raise RuntimeError("device status after warm-up is not OK")
+
+    n_ev = 6
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device() if "CUDA_VISIBLE_DEVICES" not in os.environ else local_rank) as clk:
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for i in range(args.steps):
+                step.run(stream, evs[i])
+            t1.record(stream)
+        stream.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = t0.elapsed_time(t1)
+    if world > 1:
+        import torch.distributed as dist
+        tt = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    status = lsa.dit_device_status(clear=True)
+
+    full_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    chunk_ms = [e[1].elapsed_time(e[2]) for e in evs] if step.bounds else []
+    merge_ms = [e[2].elapsed_time(e[3]) for e in evs] if step.bounds else []
+    fp8_ms = [e[4].elapsed_time(e[5]) for e in evs] if fp8 else []
+
+    # end to end through the C ABI with host buffers: pinned H2D of Q, K, V, the step, D2H of
+    # the outputs, all inside the timed region
+    e2e = run_e2e(args, lsa, step, data, stream, dev)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peaks_src = load_peaks()
+    total_flops = step.flops * args.steps * world
+    value = total_flops / (elapsed_ms * 1e-3) / 1e12
+    avg_full = statistics.mean(full_ms)
+    achieved = w.flops / (avg_full * 1e-3) / 1e12
+    peak = peaks["bf16_tflops"]
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(elapsed_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) rounded to bf16; no weights involved)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D, "scale": w.scale,
+                   "n_chunks": w.n_chunks, "fp8_variant": fp8,
+                   "step": "dit_attn_fwd + %d x dit_attn_fwd_chunk + dit_attn_merge%s" % (
+                       len(step.bounds), " + 3 x dit_quant_fp8 + dit_attn_fwd(e4m3)" if fp8 else ""),
+                   "l2": "no flush: Q/K/V (%.0f MB) exceed the 126 MB L2" % (3 * w.B * w.H * w.S * w.D * 2 / 1e6),
+                   "parallelism": "replicas%d" % world},
+        "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (dit_attn_fwd)",
+                     "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                     "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
+                     "traffic": profiled_traffic(),
+                     "algorithmic_bytes": 4 * w.B * w.H * w.S * w.D * 2 + w.B * w.H * w.S * 4},
+        "phases_ms": {"full_fwd": round(avg_full, 4),
+                      "chunks": round(statistics.mean(chunk_ms), 4) if chunk_ms else None,
+                      "merge": round(statistics.mean(merge_ms), 4) if merge_ms else None,
+                      "fp8_fwd": round(statistics.mean(fp8_ms), 4) if fp8_ms else None},
+        "gpu_launches": step.launches * args.steps,
+        "device_status": status,
+    }
+    if merge_ms:
+        n = len(step.bounds)
+        mbytes = (n * (w.B * w.H * w.S * (w.D * 4 + 4)) + w.B * w.H * w.S * (w.D * 2 + 4))
+        gbs = mbytes / (statistics.mean(merge_ms) * 1e-3) / 1e9
+        line["merge_roofline"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                                  "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                  "algorithmic_bytes": mbytes}
+    if fp8_ms:
+        line["fp8_fwd_tflops"] = round(w.flops / (statistics.mean(fp8_ms) * 1e-3) / 1e12, 2)
+    line["clocks"] = clk.summary()
+    line["e2e"] = e2e
+    if world == 1 and not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, lsa, step, data, stream, dev):
+    import torch
+    w = step.w
+    host_in = [torch.from_numpy(data[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"]
+    host_out = torch.empty(step.out.shape, dtype=torch.bfloat16).pin_memory()
+    host_lse = torch.empty(step.lse.shape, dtype=torch.float32).pin_memory()
+    outs = [(host_out, step.out), (host_lse, step.lse)]
+    if step.bounds:
+        host_mout = torch.empty(step.mout.shape, dtype=torch.bfloat16).pin_memory()
+        host_mlse = torch.empty(step.mlse.shape, dtype=torch.float32).pin_memory()
+        outs += [(host_mout, step.mout), (host_mlse, step.mlse)]
+    if step.fp8:
+        host_o8 = torch.empty(step.out8.shape, dtype=torch.bfloat16).pin_memory()
+        outs += [(host_o8, step.out8)]
+    n_steps = max(3, min(args.steps, 10))
+
+    def one():
+        for h, d in zip(host_in, (step.q, step.k, step.v)):
+            d.copy_(h, non_blocking=True)
+        step.run(stream)
+        for h, d in outs:
+            h.copy_(d, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        one()
+        stream.synchronize()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(n_steps):
+            one()
+        t1.record(stream)
+    stream.synchronize()
+    ms = t0.elapsed_time(t1) / n_steps
+    bi = sum(h.numel() * h.element_size() for h in host_in)
+    bo = sum(h.numel() * h.element_size() for h, _ in outs)
+    return {"value": round(step.flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
+            "steps": n_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+
+
+# ----------------------------------------------------------------------------- oracle (CPU)
+def cpu_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w, data, rows, heads):
+    """Time the fp64 oracle on the given query rows of the given heads (full KV range)."""
+    import oracle
+    q = data["q"][:, heads]
+    k = data["k"][:, heads]
+    v = data["v"][:, heads]
+    t = time.perf_counter()
+    oracle.attention(q, k, v, w.scale, rows=rows)
+    dt = time.perf_counter() - t
+    flops = 4.0 * w.B * len(heads) * len(rows) * w.S * w.D
+    return flops, dt
+
+
+def cpu_baseline(w, seconds: float):
+    """The oracle as it stands, on a bounded sample of the workload sized to ~`seconds`."""
+    data = make_qkv(w)
+    heads = list(range(w.H))
+    rows = list(range(0, min(w.S, 64)))
+    flops, dt = oracle_sample(w, data, rows, heads[:1])
+    per_row_head = dt / len(rows)
+    n_rows = int(max(64, min(w.S, seconds / max(per_row_head * w.H, 1e-9))))
+    rows = list(range(n_rows))
+    flops, dt = oracle_sample(w, data, rows, heads)
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"fp64 oracle, {w.B} batch x {w.H} heads x first {n_rows} query rows x all {w.S} keys "
+                      f"of {w.name} ({flops:.3e} FLOP)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    data = make_qkv(w)
+    heads = list(range(w.H))
+    # size one step to ~ args.ref_step_seconds of CPU work
+    _, dt = oracle_sample(w, data, list(range(32)), [0])
+    n_rows = int(max(16, min(w.S, args.ref_step_seconds / max(dt / 32 * w.H, 1e-9))))
+    rows = list(range(n_rows))
+    for _ in range(args.warmup):
+        oracle_sample(w, data, rows[:16], heads[:1])
+    times, flops = [], 0.0
+    for _ in range(args.steps):
+        f, dt = oracle_sample(w, data, rows, heads)
+        times.append(dt)
+        flops = f
+    total = sum(times)
+    value = flops * args.steps / total / 1e12
+    sample = (f"per step: fp64 oracle on {w.B} batch x {w.H} heads x first {n_rows} query rows x all {w.S} keys "
+              f"of {w.name} ({flops:.3e} FLOP)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(total / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) rounded to bf16)",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D, "scale": w.scale},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="flux_2048", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline sample")
+    ap.add_argument("--ref-step-seconds", type=float, default=6.0, help="CPU work per --impl reference step")
+    ap.add_argument("--skip-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, local_rank, world = rank_info()
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, local_rank, world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,154 @@
+/*
+ * dit_attn.h - C ABI of a B200 (sm_100a) library for DiT joint self-attention.
+ *
+ * What the library computes
+ * -------------------------
+ * The attention at the heart of a diffusion-transformer (DiT) block: image or video patch
+ * tokens concatenated with text tokens, every token attending to every token (no causal
+ * mask, no padding mask, no KV cache).  The source pages describe DiT inference as
+ * prefill-like and compute-bound from start to finish, with sequences of many thousands of
+ * tokens (xDiT overview page, sections 1 and 2.1-2.2).  For each batch b, head h and query
+ * row i, over the keys j of a range [k0, k1):
+ *
+ *     out_i = sum_j softmax_j(scale * q_i . k_j) v_j
+ *     lse_i = log sum_j exp(scale * q_i . k_j)          (natural log)
+ *
+ * Partial results over disjoint key ranges are combined exactly by dit_attn_merge, the
+ * combine step that the USP "Ring" dimension relies on (xDiT overview page, section 3.2.2:
+ * the sequence is split into blocks passed around a ring; the xDiT docs page exposes it as
+ * --ring_degree).  An FP8-E4M3 input variant follows the FP8 attention backend named on the
+ * AMD ROCm summary page (--attention_backend aiter_flydsl_fp8; "FP8 may change outputs").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensors are dense row-major [B, H, S, D] (D innermost, stride 1); LSE arrays are fp32
+ *    [B, H, S].  D must be 64 or 128.
+ *  - Every tensor pointer is a DEVICE pointer on the current CUDA device, 16-byte aligned
+ *    (LSE pointers 4-byte aligned).  The caller owns all buffers; the library never
+ *    allocates, frees or keeps device memory, and never synchronises the stream.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is enqueued on it
+ *    and the call returns immediately; the calls are therefore usable inside CUDA-graph
+ *    capture.
+ *  - Return value: DIT_OK or a DIT_ERR_* code.  Argument errors are detected on the host
+ *    before anything is enqueued.  A failed launch returns DIT_ERR_CUDA.  Errors that can
+ *    only arise on the device (a bounded wait that ran out, DIT_ERR_TIMEOUT) are recorded
+ *    in a device status word read by dit_device_status().
+ *  - Outputs must not overlap inputs.
+ *  - Thread-safe: calls on different streams or host threads may run concurrently.
+ */
+#ifndef DIT_ATTN_H
+#define DIT_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* element types */
+#define DIT_BF16 0     /* bfloat16 */
+#define DIT_FP8_E4M3 1 /* FP8 E4M3 ("fn": no infinities, max 448) with a per-tensor descale */
+#define DIT_FP32 2     /* float32 (outputs only) */
+
+/* status codes */
+#define DIT_OK 0
+#define DIT_ERR_INVALID_ARG 1 /* null pointer, bad size, bad range, overlapping buffers */
+#define DIT_ERR_UNSUPPORTED 2 /* valid but not built: D not in {64,128}, FP8 with D != 128 */
+#define DIT_ERR_MISALIGNED 3  /* a pointer breaks the alignment rule above */
+#define DIT_ERR_CUDA 4        /* a CUDA runtime/driver call or a launch failed */
+#define DIT_ERR_TIMEOUT 5     /* device side: a bounded wait inside a kernel ran out */
+
+/*
+ * dit_attn_fwd - full attention forward over all S keys.
+ *
+ *   q, k, v   [B,H,S,D] inputs, bf16 (dtype = DIT_BF16) or E4M3 codes (DIT_FP8_E4M3).
+ *   out       [B,H,S,D] bf16 output.
+ *   lse       [B,H,S] fp32 natural-log LSE, or NULL to skip it.
+ *   scale     softmax scale (finite, > 0), usually 1/sqrt(D).
+ *   descale_qkv  DIT_FP8_E4M3 only: device pointer to 3 floats {descale_q, descale_k,
+ *             descale_v}; the real input is code * descale (see dit_quant_fp8).  NULL for bf16.
+ *
+ * Same as dit_attn_fwd_chunk(q,k,v,out,lse,B,H,S,S,D,0,S,scale,dtype,DIT_BF16,descale,stream).
+ */
+int dit_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                 int S, int D, float scale, int dtype, const float* descale_qkv, void* stream);
+
+/*
+ * dit_attn_fwd_chunk - attention of S_q queries against the keys k0 <= j < k1 of a
+ * [B,H,S_kv,D] K/V pair: one ring step of the USP Ring dimension, all on one GPU.
+ *
+ *   q         [B,H,S_q,D];  k, v  [B,H,S_kv,D] (full tensors; the range selects rows).
+ *   out       [B,H,S_q,D], out_dtype DIT_BF16 or DIT_FP32 (fp32 keeps partials exact
+ *             enough for a later merge).
+ *   lse       [B,H,S_q] fp32, or NULL.
+ *   0 <= k0 <= k1 <= S_kv.  k0 == k1 (an empty range) writes out = 0 and lse = -inf.
+ */
+int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int H, int S_q, int S_kv, int D, int k0, int k1, float scale, int dtype,
+                       int out_dtype, const float* descale_qkv, void* stream);
+
+/*
+ * dit_attn_merge - exact log-sum-exp combination of n_chunks partials (out_c, lse_c):
+ *     M = max_c lse_c, w_c = exp(lse_c - M), L = sum_c w_c,
+ *     lse = M + log L, out = sum_c (w_c / L) out_c;  all lse_c = -inf -> out = 0, lse = -inf.
+ *
+ *   outs      HOST array of n_chunks DEVICE pointers, each [B,H,S,D] of in_dtype
+ *             (DIT_BF16 or DIT_FP32).
+ *   lses      HOST array of n_chunks DEVICE pointers, each [B,H,S] fp32.
+ *   n_chunks  1..16.
+ *   out       [B,H,S,D] of out_dtype (DIT_BF16 or DIT_FP32);  lse [B,H,S] fp32 or NULL.
+ *   The host arrays are read during the call only.
+ */
+int dit_attn_merge(const void* const* outs, const float* const* lses, int n_chunks, void* out,
+                   float* lse, int B, int H, int S, int D, int in_dtype, int out_dtype,
+                   void* stream);
+
+/*
+ * dit_quant_fp8 - per-tensor absmax quantisation of n bf16 values to E4M3:
+ *     amax = max|x|, descale = amax / 448 (1 if amax = 0), x_fp8 = rn_satfinite(x / descale)
+ * with IEEE fp32 division.  The FP8 scaling scheme is not given by the pages; this is the
+ * plain per-tensor reading of their FP8 backend.
+ *
+ *   x_bf16    n bf16 values (16-byte aligned);  x_fp8  n bytes (16-byte aligned).
+ *   descale   device pointer to 1 float (written).
+ *   workspace device scratch of at least dit_quant_fp8_workspace_bytes(n) bytes, 4-byte
+ *             aligned, owned by the caller; its contents on entry do not matter.
+ */
+size_t dit_quant_fp8_workspace_bytes(long long n);
+int dit_quant_fp8(const void* x_bf16, void* x_fp8, float* descale, long long n, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
+ * dit_device_status - synchronises the current device, then reads the device status word
+ * into *status: DIT_OK, or DIT_ERR_TIMEOUT | (site << 8) when a bounded wait inside a
+ * kernel ran out (the kernel then wound down without hanging; its outputs are invalid).
+ * clear != 0 resets the word to DIT_OK afterwards.  Returns DIT_ERR_CUDA if the device
+ * cannot be synchronised or read.
+ */
+int dit_device_status(int* status, int clear);
+
+/*
+ * dit_set_wait_timeout_us - process-wide limit for every bounded wait inside the kernels
+ * (default 1,000,000 us).  A healthy kernel waits microseconds; the limit only matters
+ * if the pipeline is broken.  0 restores the default.
+ */
+int dit_set_wait_timeout_us(unsigned long long timeout_us);
+
+/*
+ * dit_selftest_wait_timeout - enqueues a one-thread kernel that waits on a barrier nothing
+ * ever arrives at, with the given limit, so the caller can check that the bounded wait
+ * gives up and that dit_device_status() then reports DIT_ERR_TIMEOUT.
+ */
+int dit_selftest_wait_timeout(unsigned long long timeout_us, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* dit_status_str(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int dit_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DIT_ATTN_H */

@@ -1,0 +1,200 @@
+"""Python binding of the DiT joint-attention library for B200 (sm_100a).
+
+Argument marshalling only: every computation runs in the CUDA kernels of
+``libdit_attn.so`` (built in-tree by ``long_sequence_attention_b200.build``).  The C
+functions keep their names here (``dit_attn_fwd``, ``dit_attn_fwd_chunk``,
+``dit_attn_merge``, ``dit_quant_fp8`` ...); tensors may be passed as torch CUDA tensors or
+as raw device addresses (ints).  A non-zero status raises ``DitError``.
+
+Importing this package fails loudly (ImportError) when the library has not been built:
+there is no fallback implementation.
+
+The few ``attention`` / ``attention_chunk`` / ``merge`` / ``quantize_fp8`` helpers below
+only allocate outputs with torch and call the C entry points.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdit_attn.so")
+
+DIT_BF16, DIT_FP8_E4M3, DIT_FP32 = 0, 1, 2
+DIT_OK, DIT_ERR_INVALID_ARG, DIT_ERR_UNSUPPORTED, DIT_ERR_MISALIGNED, DIT_ERR_CUDA, DIT_ERR_TIMEOUT = range(6)
+
+
+class DitError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {status_str(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_sequence_attention_b200.build` "
+                          "(nvcc, sm_100a). There is no CPU fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
+    sz, ull = ctypes.c_size_t, ctypes.c_ulonglong
+    lib.dit_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
+    lib.dit_attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp, vp]
+    lib.dit_attn_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, vp, vp, i, i, i, i, i, i, vp]
+    lib.dit_quant_fp8_workspace_bytes.argtypes = [ll]
+    lib.dit_quant_fp8_workspace_bytes.restype = sz
+    lib.dit_quant_fp8.argtypes = [vp, vp, vp, ll, vp, sz, vp]
+    lib.dit_device_status.argtypes = [ctypes.POINTER(i), i]
+    lib.dit_set_wait_timeout_us.argtypes = [ull]
+    lib.dit_selftest_wait_timeout.argtypes = [ull, vp]
+    lib.dit_status_str.argtypes = [i]
+    lib.dit_status_str.restype = ctypes.c_char_p
+    lib.dit_version.argtypes = []
+    for name in ("dit_attn_fwd", "dit_attn_fwd_chunk", "dit_attn_merge", "dit_quant_fp8", "dit_device_status",
+                 "dit_set_wait_timeout_us", "dit_selftest_wait_timeout", "dit_version"):
+        getattr(lib, name).restype = ctypes.c_int
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.dit_status_str(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != DIT_OK:
+        raise DitError(rc, where)
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# --------------------------------------------------------------------------- C entry points
+
+def dit_attn_fwd(q, k, v, out, lse, B: int, H: int, S: int, D: int, scale: float,
+                 dtype: int = DIT_BF16, descale_qkv=None, stream=None) -> None:
+    _check(lib.dit_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D, float(scale),
+                            dtype, _ptr(descale_qkv), _stream(stream)), "dit_attn_fwd")
+
+
+def dit_attn_fwd_chunk(q, k, v, out, lse, B: int, H: int, S_q: int, S_kv: int, D: int, k0: int, k1: int,
+                       scale: float, dtype: int = DIT_BF16, out_dtype: int = DIT_FP32, descale_qkv=None,
+                       stream=None) -> None:
+    _check(lib.dit_attn_fwd_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S_q, S_kv, D, k0, k1,
+                                  float(scale), dtype, out_dtype, _ptr(descale_qkv), _stream(stream)),
+           "dit_attn_fwd_chunk")
+
+
+def dit_attn_merge(outs: Sequence, lses: Sequence, out, lse, B: int, H: int, S: int, D: int,
+                   in_dtype: int = DIT_FP32, out_dtype: int = DIT_BF16, stream=None) -> None:
+    n = len(outs)
+    arr_o = (ctypes.c_void_p * n)(*[_ptr(o) for o in outs])
+    arr_l = (ctypes.c_void_p * n)(*[_ptr(x) for x in lses])
+    _check(lib.dit_attn_merge(arr_o, arr_l, n, _ptr(out), _ptr(lse), B, H, S, D, in_dtype, out_dtype,
+                              _stream(stream)), "dit_attn_merge")
+
+
+def dit_quant_fp8_workspace_bytes(n: int) -> int:
+    return int(lib.dit_quant_fp8_workspace_bytes(int(n)))
+
+
+def dit_quant_fp8(x_bf16, x_fp8, descale, n: int, workspace, workspace_bytes: int, stream=None) -> None:
+    _check(lib.dit_quant_fp8(_ptr(x_bf16), _ptr(x_fp8), _ptr(descale), int(n), _ptr(workspace),
+                             int(workspace_bytes), _stream(stream)), "dit_quant_fp8")
+
+
+def dit_device_status(clear: bool = True) -> int:
+    st = ctypes.c_int(0)
+    _check(lib.dit_device_status(ctypes.byref(st), 1 if clear else 0), "dit_device_status")
+    return st.value
+
+
+def dit_set_wait_timeout_us(us: int) -> None:
+    _check(lib.dit_set_wait_timeout_us(int(us)), "dit_set_wait_timeout_us")
+
+
+def dit_selftest_wait_timeout(timeout_us: int, stream=None) -> None:
+    _check(lib.dit_selftest_wait_timeout(int(timeout_us), _stream(stream)), "dit_selftest_wait_timeout")
+
+
+def dit_version() -> int:
+    return int(lib.dit_version())
+
+
+# --------------------------------------------------------------------------- torch helpers
+
+def _dims(q):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, H, S, D] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def attention(q, k, v, scale: Optional[float] = None, with_lse: bool = True, descale_qkv=None,
+              stream=None) -> Tuple[object, Optional[object]]:
+    """out (bf16) and lse (fp32) of full attention; q/k/v bf16 or uint8 E4M3 codes."""
+    import torch
+    B, H, S, D = _dims(q)
+    fp8 = q.dtype == torch.uint8
+    scale = (1.0 / D ** 0.5) if scale is None else scale
+    out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=q.device)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if with_lse else None
+    dit_attn_fwd(q, k, v, out, lse, B, H, S, D, scale, DIT_FP8_E4M3 if fp8 else DIT_BF16, descale_qkv, stream)
+    return out, lse
+
+
+def attention_chunk(q, k, v, k0: int, k1: int, scale: Optional[float] = None, out_dtype=None,
+                    descale_qkv=None, stream=None):
+    """Partial (out, lse) over keys [k0, k1); out fp32 unless out_dtype is torch.bfloat16."""
+    import torch
+    B, H, S_q, D = _dims(q)
+    S_kv = int(k.shape[2])
+    fp8 = q.dtype == torch.uint8
+    scale = (1.0 / D ** 0.5) if scale is None else scale
+    od = torch.float32 if out_dtype is None else out_dtype
+    out = torch.empty((B, H, S_q, D), dtype=od, device=q.device)
+    lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q.device)
+    dit_attn_fwd_chunk(q, k, v, out, lse, B, H, S_q, S_kv, D, k0, k1, scale,
+                       DIT_FP8_E4M3 if fp8 else DIT_BF16, DIT_FP32 if od == torch.float32 else DIT_BF16,
+                       descale_qkv, stream)
+    return out, lse
+
+
+def merge(outs: Sequence, lses: Sequence, out_dtype=None, stream=None):
+    """Merged (out, lse) of chunk partials; out bf16 unless out_dtype is torch.float32."""
+    import torch
+    B, H, S, D = _dims(outs[0])
+    od = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((B, H, S, D), dtype=od, device=outs[0].device)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=outs[0].device)
+    in_dt = DIT_FP32 if outs[0].dtype == torch.float32 else DIT_BF16
+    dit_attn_merge(outs, lses, out, lse, B, H, S, D, in_dt, DIT_FP32 if od == torch.float32 else DIT_BF16, stream)
+    return out, lse
+
+
+def quantize_fp8(x, stream=None):
+    """(codes uint8 same shape, descale fp32 [1]) of a bf16 tensor; per-tensor absmax scale."""
+    import torch
+    n = x.numel()
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    descale = torch.empty((1,), dtype=torch.float32, device=x.device)
+    ws_bytes = dit_quant_fp8_workspace_bytes(n)
+    ws = torch.empty((ws_bytes // 4,), dtype=torch.float32, device=x.device)
+    dit_quant_fp8(x, codes, descale, n, ws, ws_bytes, stream)
+    return codes, descale

@@ -1,0 +1,439 @@
+// Flash-style forward attention for sm_100a: TMA-staged Q/K/V tiles, tcgen05 MMAs with
+// S = Q K^T and O += P V accumulated in TMEM, online softmax in registers.
+//
+// What it computes (joint image+text self-attention of a DiT block; the xDiT overview page,
+// section 2.1, describes DiT inference as prefill-like and compute-bound, with every token
+// attending to every token and no KV cache): for each (b, h) and query row i, over the keys
+// k0 <= j < k1,
+//     out_i = sum_j softmax_j(scale * q_i . k_j) v_j,   lse_i = log sum_j exp(scale * q_i . k_j).
+// The KV-range form is the per-block step of the USP "Ring" dimension (xDiT overview,
+// section 3.2.2): a ring step attends the local queries to one block of keys and the partial
+// results are combined afterwards by the log-sum-exp merge (merge.cuh).
+//
+// Work unit: one CTA per (b, h, 256 query rows) = two 128-row Q tiles that ping-pong, so the
+// exponentials of one tile overlap the tensor-core work of the other.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp  8    MMA issuer (one thread issues every tcgen05.mma and commit)
+//   warp  9    TMA producer (Q once, then a ring of K stages and a ring of V stages)
+//
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).  P (bf16 or
+// e4m3) is written over the first columns of S and read from TMEM by the P.V MMA.
+//
+// Ordering facts the pipeline relies on:
+//   * MMAs issued by one thread execute in order, and tcgen05.commit fires only when every
+//     earlier MMA of that thread is done.  The MMA thread issues  PV_t(j-1)  before  S_t(j)
+//     for each tile t, so when the softmax warpgroup sees S_t(j) ready, PV_t(j-1) has also
+//     finished: O_t is quiescent and the warpgroup may rescale it in place before it
+//     publishes P_t(j).  It also means S_t(j) never overwrites P_t(j-1) while it is read.
+//   * Max tracking is lazy: a row keeps its running max m_use until a new tile raises the
+//     max by more than kRescaleLog2 (in log2 units); until then p = 2^(c(x - m_use)) may
+//     exceed 1 but stays <= 2^kRescaleLog2, which bf16 / fp32 hold exactly enough.  The final
+//     normalisation uses the same m_use for l and O, so the result is exact up to rounding.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "ptx.cuh"
+
+namespace dit {
+
+struct AttnParams {
+  int B, H, S_q, S_kv;
+  int k0, k1;
+  float scale;             // softmax scale applied to q.k
+  const float* descale;    // e4m3 path: device pointer to {descale_q, descale_k, descale_v}
+  void* out;               // [B,H,S_q,D] bf16 or fp32
+  float* lse;              // [B,H,S_q] natural-log LSE, may be null
+  int out_fp32;
+  unsigned long long timeout_ns;
+};
+
+// exp2 on the FMA pipe for x <= 2^7: x = n + f with n = rint(x), f in [-1/2, 1/2];
+// 2^f by a degree-3 polynomial (minimax in relative error, max 7.5e-5; coefficients from
+// fit_exp2_poly.py); 2^n by adding n to the exponent field.  x is clamped at -125 so the
+// exponent never underflows (2^-125 stands in for 0; it only ever multiplies V values).
+__device__ __forceinline__ float exp2_fma(float x) {
+  x = fmaxf(x, -125.0f);
+  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds x to an integer
+  const float t = x + magic;
+  const float n = t - magic;
+  const float f = x - n;
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  // low bits of t hold n (two's complement); shifting them into the exponent field adds n
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+template <int D, bool FP8>
+struct AttnCfg {
+  static constexpr int kBM = 128;                       // query rows per tile
+  static constexpr int kBN = 128;                       // keys per KV tile
+  static constexpr int kElem = FP8 ? 1 : 2;             // bytes per element
+  static constexpr int kRowBytes = D * kElem;           // bytes of one row
+  static constexpr int kBlkBytes = 128 * 128;           // one 128-row x 128-byte swizzle block
+  static constexpr int kNBlk = kRowBytes / 128;         // 128-byte column blocks per row
+  static constexpr int kTileBytes = 128 * kRowBytes;
+  static constexpr int kBoxInner = 128 / kElem;         // TMA box width in elements
+  static constexpr int kKStages = (kTileBytes >= 32768) ? 2 : 4;
+  static constexpr int kVStages = kKStages;
+  static constexpr int kUmmaK = 32 / kElem;             // K per MMA instruction (32 bytes)
+  static constexpr int kQKSteps = kRowBytes / 32;       // MMAs per S tile
+  static constexpr int kPVSteps = kBN / kUmmaK;         // MMAs per P.V
+  static constexpr int kThreads = 320;
+  static constexpr int kMmaWarp = 8;
+  static constexpr int kTmaWarp = 9;
+  static constexpr int kTmemCols = 512;
+  static constexpr int kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + D;
+  // P is kept <= 2^(kRescaleLog2 + kPShift); for e4m3 (max 448) it is shifted up so that
+  // most probabilities are normal numbers rather than subnormals.
+  static constexpr float kRescaleLog2 = FP8 ? 4.0f : 8.0f;
+  static constexpr float kPShift = FP8 ? 4.0f : 0.0f;
+
+  // shared memory layout (offsets from a 1024-byte aligned base)
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kKStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
+  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(!FP8 || D == 128, "e4m3 path is built for D = 128");
+};
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(320, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+  using C = AttnCfg<D, FP8>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* bar_q_full = bars;
+  uint64_t* bar_k_full = bars + 1;
+  uint64_t* bar_k_empty = bar_k_full + C::kKStages;
+  uint64_t* bar_v_full = bar_k_empty + C::kKStages;
+  uint64_t* bar_v_empty = bar_v_full + C::kVStages;
+  uint64_t* bar_s_full = bar_v_empty + C::kVStages;   // [2]
+  uint64_t* bar_p_full = bar_s_full + 2;              // [2]
+  uint64_t* bar_o_final = bar_p_full + 2;             // [2]
+  uint64_t* bar_drain = bar_o_final + 2;              // [1]
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.z * p.H + blockIdx.y;
+  const int q_start = blockIdx.x * (2 * C::kBM);
+  const int n_kv = (p.k1 - p.k0 + C::kBN - 1) / C::kBN;   // >= 1 (empty ranges never launch)
+  const uint64_t tmo = p.timeout_ns;
+
+  if (threadIdx.x == C::kTmaWarp * 32) {
+    mbar_init(bar_q_full, 1);
+    for (int s = 0; s < C::kKStages; ++s) { mbar_init(bar_k_full + s, 1); mbar_init(bar_k_empty + s, 1); }
+    for (int s = 0; s < C::kVStages; ++s) { mbar_init(bar_v_full + s, 1); mbar_init(bar_v_empty + s, 1); }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + t, 1);
+      mbar_init(bar_p_full + t, 4);
+      mbar_init(bar_o_final + t, 1);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  uint8_t* sQ = smem + C::kOffQ;
+  uint8_t* sK = smem + C::kOffK;
+  uint8_t* sV = smem + C::kOffV;
+
+  if (warp == C::kTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int b = 0; b < C::kNBlk; ++b)
+          tma_load_3d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
+                      q_start + t * C::kBM, bh);
+      int k_issued = 0, v_issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int kv_row = p.k0 + j * C::kBN;
+        const int ks = j % C::kKStages;
+        if (j >= C::kKStages &&
+            !mbar_wait(bar_k_empty + ks, ((j / C::kKStages) + 1) & 1, abort_flag, tmo, 1))
+          break;
+        mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
+        for (int b = 0; b < C::kNBlk; ++b)
+          tma_load_3d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
+                      b * C::kBoxInner, kv_row, bh);
+        k_issued = j + 1;
+        const int vs = j % C::kVStages;
+        if (j >= C::kVStages &&
+            !mbar_wait(bar_v_empty + vs, ((j / C::kVStages) + 1) & 1, abort_flag, tmo, 2))
+          break;
+        mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
+        for (int b = 0; b < C::kNBlk; ++b)
+          tma_load_3d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
+                      b * C::kBoxInner, kv_row, bh);
+        v_issued = j + 1;
+      }
+      // Drain: the last load armed on every stage must land before the CTA may exit
+      // (a no-op in a healthy run, where the consumers already waited for all of them).
+      mbar_wait_drain(bar_q_full, 0, tmo);
+      for (int s = 0; s < C::kKStages; ++s) {
+        const int last = s + ((k_issued - 1 - s) / C::kKStages) * C::kKStages;
+        if (k_issued > s) mbar_wait_drain(bar_k_full + s, (last / C::kKStages) & 1, tmo);
+      }
+      for (int s = 0; s < C::kVStages; ++s) {
+        const int last = s + ((v_issued - 1 - s) / C::kVStages) * C::kVStages;
+        if (v_issued > s) mbar_wait_drain(bar_v_full + s, (last / C::kVStages) & 1, tmo);
+      }
+    }
+  } else if (warp == C::kMmaWarp) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t fmt = FP8 ? 0u : 1u;
+      constexpr uint32_t id_s = instr_desc(fmt, false, 128, C::kBN);
+      constexpr uint32_t id_o = instr_desc(fmt, true, 128, D);
+      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+
+      auto issue_s = [&](int t, int ks) {
+        const uint32_t a0 = q_addr + t * C::kTileBytes;
+        const uint32_t b0 = k_addr + ks * C::kTileBytes;
+        const uint32_t d = tmem_base + (t ? C::kColS1 : C::kColS0);
+#pragma unroll
+        for (int kk = 0; kk < C::kQKSteps; ++kk) {
+          const uint32_t off = (kk * 32 / 128) * C::kBlkBytes + (kk * 32) % 128;
+          const uint64_t ad = smem_desc_sw128(a0 + off, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(b0 + off, 16, 1024);
+          if constexpr (FP8) mma_f8_ss(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          else mma_f16_ss(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int vs, bool acc) {
+        const uint32_t b0 = v_addr + vs * C::kTileBytes;
+        const uint32_t a_tm = tmem_base + (t ? C::kColS1 : C::kColS0);
+        const uint32_t d = tmem_base + (t ? C::kColO1 : C::kColO0);
+#pragma unroll
+        for (int kk = 0; kk < C::kPVSteps; ++kk) {
+          // V tile is [kv rows][D] with D contiguous: MN-major B operand.  One MMA covers
+          // kUmmaK kv rows (groups of 8 rows 1024 bytes apart) and all of D (64-element,
+          // 128-byte atoms kBlkBytes apart).
+          const uint64_t bd = smem_desc_sw128(b0 + kk * C::kUmmaK * 128, C::kBlkBytes, 1024);
+          const uint32_t acc_flag = (acc || kk > 0) ? 1u : 0u;
+          if constexpr (FP8) mma_f8_ts(d, a_tm + kk * 8, bd, id_o, acc_flag);
+          else mma_f16_ts(d, a_tm + kk * 8, bd, id_o, acc_flag);
+        }
+      };
+
+      bool ok = mbar_wait(bar_q_full, 0, abort_flag, tmo, 3);
+      if (ok) tc_fence_after();
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int ks = j % C::kKStages;
+        if (!(ok = mbar_wait(bar_k_full + ks, (j / C::kKStages) & 1, abort_flag, tmo, 4))) break;
+        tc_fence_after();
+        const int jp = j - 1, vs = (j - 1) % C::kVStages;
+        if (j > 0) {
+          if (!(ok = mbar_wait(bar_v_full + vs, (jp / C::kVStages) & 1, abort_flag, tmo, 5))) break;
+          if (!(ok = mbar_wait(bar_p_full + 0, jp & 1, abort_flag, tmo, 6))) break;
+          tc_fence_after();
+          issue_pv(0, vs, jp > 0);
+        }
+        issue_s(0, ks);
+        tc_commit(bar_s_full + 0);
+        if (j > 0) {
+          if (!(ok = mbar_wait(bar_p_full + 1, jp & 1, abort_flag, tmo, 7))) break;
+          tc_fence_after();
+          issue_pv(1, vs, jp > 0);
+          tc_commit(bar_v_empty + vs);
+        }
+        issue_s(1, ks);
+        tc_commit(bar_s_full + 1);
+        tc_commit(bar_k_empty + ks);
+      }
+      if (ok) {
+        const int jl = n_kv - 1, vs = jl % C::kVStages;
+        ok = mbar_wait(bar_v_full + vs, (jl / C::kVStages) & 1, abort_flag, tmo, 8);
+        if (ok) ok = mbar_wait(bar_p_full + 0, jl & 1, abort_flag, tmo, 9);
+        if (ok) {
+          tc_fence_after();
+          issue_pv(0, vs, jl > 0);
+          tc_commit(bar_o_final + 0);
+          ok = mbar_wait(bar_p_full + 1, jl & 1, abort_flag, tmo, 10);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_pv(1, vs, jl > 0);
+          tc_commit(bar_o_final + 1);
+        }
+      }
+      // Every MMA this thread issued must finish before TMEM is released.
+      tc_commit(bar_drain);
+      mbar_wait_drain(bar_drain, 0, tmo);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;                // Q tile of this warpgroup
+    const int quad = warp & 3;              // TMEM lane quadrant of this warp
+    const int row = quad * 32 + lane;       // row within the tile == TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tS = tmem_base + lane_off + (t ? C::kColS1 : C::kColS0);
+    const uint32_t tO = tmem_base + lane_off + (t ? C::kColO1 : C::kColO0);
+
+    float dq = 1.0f, dk = 1.0f, dv = 1.0f;
+    if constexpr (FP8) { dq = p.descale[0]; dk = p.descale[1]; dv = p.descale[2]; }
+    const float scale_eff = p.scale * dq * dk;                 // natural-log units per raw score
+    const float cl = scale_eff * 1.4426950408889634f;          // log2 units per raw score
+    float m_use = -INFINITY;                                   // running (lazy) max, raw units
+    float l = 0.0f;
+    bool ok = true;
+
+    for (int j = 0; j < n_kv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag, tmo, 11 + t));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld128_sync(tS, s);
+      const int valid = p.k1 - (p.k0 + j * C::kBN);
+      if (valid < C::kBN) {
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (c >= valid) s[c] = 0xFF800000u;                  // -inf
+      }
+      float mx[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(s[c]);
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
+      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      const float m_new = fmaxf(m_use, mt);
+      const bool need = (m_new - m_use) * cl > C::kRescaleLog2;   // true on the first tile
+      float alpha = 1.0f;
+      if (need) {
+        alpha = ex2_approx((m_use - m_new) * cl);              // 0 when m_use = -inf
+        m_use = m_new;
+      }
+      const float mc = m_use * cl - C::kPShift;
+      float sum[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pa[32], pb[32];               // P words for TMEM columns [0,32) and [32,64)
+      if constexpr (!FP8) {
+#pragma unroll
+        for (int c2 = 0; c2 < 64; ++c2) {
+          const float x0 = fmaf(__uint_as_float(s[2 * c2]), cl, -mc);
+          const float x1 = fmaf(__uint_as_float(s[2 * c2 + 1]), cl, -mc);
+          float e0, e1;
+          if ((c2 & 3) == 3) { e0 = exp2_fma(x0); e1 = exp2_fma(x1); }
+          else { e0 = ex2_approx(x0); e1 = ex2_approx(x1); }
+          sum[c2 & 3] += e0 + e1;
+          if (c2 < 32) pa[c2] = pack_bf16x2(e0, e1);
+          else pb[c2 - 32] = pack_bf16x2(e0, e1);
+        }
+        tmem_st32(tS, pa);
+        tmem_st32(tS + 32, pb);
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < 32; ++c4) {
+          float e[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float x = fmaf(__uint_as_float(s[4 * c4 + u]), cl, -mc);
+            e[u] = ((c4 & 3) == 3) ? exp2_fma(x) : ex2_approx(x);
+          }
+          sum[c4 & 3] += (e[0] + e[1]) + (e[2] + e[3]);
+          pa[c4] = pack_e4m3x4(e[0], e[1], e[2], e[3]);
+        }
+        tmem_st32(tS, pa);
+      }
+      tmem_st_wait();
+      // O_t is quiescent here (PV_t(j-1) completed before S_t(j) was signalled).
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32_sync(tO + cc * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(tO + cc * 32, o);
+        }
+        tmem_st_wait();
+      }
+      l = fmaf(l, alpha, (sum[0] + sum[1]) + (sum[2] + sum[3]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_p_full + t);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final + t, 0, abort_flag, tmo, 13 + t));
+    if (ok) {
+      tc_fence_after();
+      const int grow = q_start + t * C::kBM + row;
+      const bool store = grow < p.S_q;
+      const float inv_l = dv / l;
+      const size_t row_elem = (static_cast<size_t>(bh) * p.S_q + grow) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32_sync(tO + cc * 32, o);
+        if (store) {
+          if (p.out_fp32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_elem + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
+                                   __uint_as_float(o[4 * i + 2]) * inv_l, __uint_as_float(o[4 * i + 3]) * inv_l);
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_elem + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          }
+        }
+      }
+      if (store && p.lse != nullptr)
+        p.lse[static_cast<size_t>(bh) * p.S_q + grow] =
+            scale_eff * m_use + logf(l) - C::kPShift * 0.6931471805599453f;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// Empty KV range: out = 0, lse = -inf.
+__global__ void attn_fill_empty_kernel(void* out, float* lse, long long rows, int D, int out_fp32) {
+  const long long n = rows * D;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    if (out_fp32) static_cast<float*>(out)[i] = 0.0f;
+    else static_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16(0.0f);
+    if (lse != nullptr && i < rows) lse[i] = -INFINITY;
+  }
+}
+
+}  // namespace dit

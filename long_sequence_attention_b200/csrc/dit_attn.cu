@@ -1,0 +1,274 @@
+// C-ABI boundary of the DiT attention library: argument validation, TMA descriptor
+// construction, kernel launches and status codes.  See include/dit_attn.h for the contract.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/dit_attn.h"
+#include "attn_fwd.cuh"
+#include "merge.cuh"
+#include "quant.cuh"
+
+namespace {
+
+using namespace dit;
+
+std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry-point lookup, so the library does
+// not link libcuda directly (it loads on machines without a GPU driver).
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+// 3-D tiled map over a [B*H, S, D] tensor: box = (128 bytes of D, 128 rows, 1 head),
+// 128-byte swizzle, zero fill out of bounds (rows past S read as zeros, per head).
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return DIT_ERR_CUDA;
+  const cuuint64_t elem = fp8 ? 1 : 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem, static_cast<cuuint64_t>(S) * D * elem};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                         const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
+// Raise the dynamic shared-memory limit of a kernel once per device.
+template <typename K>
+int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load() & bit) return DIT_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return DIT_ERR_CUDA;
+  done_mask.fetch_or(bit);
+  return DIT_OK;
+}
+
+template <int D, bool FP8>
+int launch_attn(const void* q, const void* k, const void* v, const AttnParams& prm, cudaStream_t st) {
+  using C = AttnCfg<D, FP8>;
+  static std::atomic<uint64_t> attr_done{0};
+  int rc = ensure_smem_attr(attn_fwd_kernel<D, FP8>, C::kSmemBytes, attr_done);
+  if (rc != DIT_OK) return rc;
+  CUtensorMap tq, tk, tv;
+  const int BH = prm.B * prm.H;
+  if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH)) != DIT_OK) return rc;
+  if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
+  if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
+  const dim3 grid((prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM), prm.H, prm.B);
+  attn_fwd_kernel<D, FP8><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+int grid_for(long long units, int threads, int max_blocks) {
+  long long g = (units + threads - 1) / threads;
+  if (g < 1) g = 1;
+  if (g > max_blocks) g = max_blocks;
+  return static_cast<int>(g);
+}
+
+__global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, timeout_ns, 0xEE);  // nothing arrives
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                       int S_q, int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
+                       const float* descale_qkv, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || S_q < 1 || S_kv < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
+  if (k0 < 0 || k1 < k0 || k1 > S_kv) return DIT_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
+  if (dtype != DIT_BF16 && dtype != DIT_FP8_E4M3) return DIT_ERR_INVALID_ARG;
+  if (out_dtype != DIT_BF16 && out_dtype != DIT_FP32) return DIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
+  const bool fp8 = dtype == DIT_FP8_E4M3;
+  if (fp8 && D != 128) return DIT_ERR_UNSUPPORTED;
+  if (fp8 && descale_qkv == nullptr) return DIT_ERR_INVALID_ARG;
+  if (static_cast<long long>(B) * H > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return DIT_ERR_MISALIGNED;
+  if (lse != nullptr && !aligned(lse, 4)) return DIT_ERR_MISALIGNED;
+  if (descale_qkv != nullptr && !aligned(descale_qkv, 4)) return DIT_ERR_MISALIGNED;
+  const size_t in_elem = fp8 ? 1 : 2, out_elem = out_dtype == DIT_FP32 ? 4 : 2;
+  const size_t rows_q = static_cast<size_t>(B) * H * S_q, rows_kv = static_cast<size_t>(B) * H * S_kv;
+  const size_t out_bytes = rows_q * D * out_elem;
+  if (overlaps(out, out_bytes, q, rows_q * D * in_elem) || overlaps(out, out_bytes, k, rows_kv * D * in_elem) ||
+      overlaps(out, out_bytes, v, rows_kv * D * in_elem))
+    return DIT_ERR_INVALID_ARG;
+  if (lse != nullptr && (overlaps(lse, rows_q * 4, out, out_bytes) || overlaps(lse, rows_q * 4, q, rows_q * D * in_elem) ||
+                         overlaps(lse, rows_q * 4, k, rows_kv * D * in_elem) ||
+                         overlaps(lse, rows_q * 4, v, rows_kv * D * in_elem)))
+    return DIT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (k0 == k1) {
+    const long long rows = static_cast<long long>(rows_q);
+    attn_fill_empty_kernel<<<grid_for(rows * D, 256, 148 * 16), 256, 0, st>>>(out, lse, rows, D,
+                                                                               out_dtype == DIT_FP32);
+    return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+  }
+
+  AttnParams prm;
+  prm.B = B; prm.H = H; prm.S_q = S_q; prm.S_kv = S_kv; prm.k0 = k0; prm.k1 = k1;
+  prm.scale = scale;
+  prm.descale = fp8 ? descale_qkv : nullptr;
+  prm.out = out;
+  prm.lse = lse;
+  prm.out_fp32 = out_dtype == DIT_FP32;
+  prm.timeout_ns = g_timeout_ns.load();
+  if (fp8) return launch_attn<128, true>(q, k, v, prm, st);
+  if (D == 64) return launch_attn<64, false>(q, k, v, prm, st);
+  return launch_attn<128, false>(q, k, v, prm, st);
+}
+
+int dit_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S,
+                 int D, float scale, int dtype, const float* descale_qkv, void* stream) {
+  return dit_attn_fwd_chunk(q, k, v, out, lse, B, H, S, S, D, 0, S, scale, dtype, DIT_BF16, descale_qkv, stream);
+}
+
+int dit_attn_merge(const void* const* outs, const float* const* lses, int n_chunks, void* out, float* lse,
+                   int B, int H, int S, int D, int in_dtype, int out_dtype, void* stream) {
+  if (outs == nullptr || lses == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (n_chunks < 1 || n_chunks > kMaxMergeChunks) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || S < 1) return DIT_ERR_INVALID_ARG;
+  if (in_dtype != DIT_BF16 && in_dtype != DIT_FP32) return DIT_ERR_INVALID_ARG;
+  if (out_dtype != DIT_BF16 && out_dtype != DIT_FP32) return DIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(B) * H * S;
+  const size_t in_bytes = static_cast<size_t>(rows) * D * (in_dtype == DIT_FP32 ? 4 : 2);
+  const size_t out_bytes = static_cast<size_t>(rows) * D * (out_dtype == DIT_FP32 ? 4 : 2);
+  if (!aligned(out, 16) || (lse != nullptr && !aligned(lse, 4))) return DIT_ERR_MISALIGNED;
+  MergeParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  for (int c = 0; c < n_chunks; ++c) {
+    if (outs[c] == nullptr || lses[c] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned(outs[c], 16) || !aligned(lses[c], 4)) return DIT_ERR_MISALIGNED;
+    if (overlaps(out, out_bytes, outs[c], in_bytes) || overlaps(out, out_bytes, lses[c], rows * 4))
+      return DIT_ERR_INVALID_ARG;
+    if (lse != nullptr && (overlaps(lse, rows * 4, outs[c], in_bytes) || overlaps(lse, rows * 4, lses[c], rows * 4)))
+      return DIT_ERR_INVALID_ARG;
+    prm.outs[c] = outs[c];
+    prm.lses[c] = lses[c];
+  }
+  if (lse != nullptr && overlaps(lse, rows * 4, out, out_bytes)) return DIT_ERR_INVALID_ARG;
+  prm.n = n_chunks;
+  prm.out = out;
+  prm.lse = lse;
+  prm.rows = rows;
+  prm.D = D;
+  prm.in_fp32 = in_dtype == DIT_FP32;
+  prm.out_fp32 = out_dtype == DIT_FP32;
+  const long long units = rows * (D / 8);
+  lse_merge_kernel<<<grid_for(units, 256, 148 * 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+size_t dit_quant_fp8_workspace_bytes(long long n) {
+  return static_cast<size_t>(quant_blocks(n)) * sizeof(float);
+}
+
+int dit_quant_fp8(const void* x_bf16, void* x_fp8, float* descale, long long n, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  if (x_bf16 == nullptr || x_fp8 == nullptr || descale == nullptr || workspace == nullptr) return DIT_ERR_INVALID_ARG;
+  if (n < 1) return DIT_ERR_INVALID_ARG;
+  if (workspace_bytes < dit_quant_fp8_workspace_bytes(n)) return DIT_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(x_fp8, 16) || !aligned(descale, 4) || !aligned(workspace, 4))
+    return DIT_ERR_MISALIGNED;
+  if (overlaps(x_fp8, n, x_bf16, n * 2) || overlaps(workspace, workspace_bytes, x_bf16, n * 2) ||
+      overlaps(workspace, workspace_bytes, x_fp8, n) || overlaps(descale, 4, x_bf16, n * 2) ||
+      overlaps(descale, 4, x_fp8, n) || overlaps(descale, 4, workspace, workspace_bytes))
+    return DIT_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int g = quant_blocks(n);
+  float* partials = static_cast<float*>(workspace);
+  absmax_partial_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, partials);
+  if (cudaGetLastError() != cudaSuccess) return DIT_ERR_CUDA;
+  quant_e4m3_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, partials, g,
+                                                  static_cast<uint8_t*>(x_fp8), descale);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+int dit_device_status(int* status, int clear) {
+  if (status == nullptr) return DIT_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return DIT_ERR_CUDA;
+  unsigned int w = 0;
+  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return DIT_ERR_CUDA;
+  *status = static_cast<int>(w);
+  if (clear) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return DIT_ERR_CUDA;
+  }
+  return DIT_OK;
+}
+
+int dit_set_wait_timeout_us(unsigned long long timeout_us) {
+  g_timeout_ns.store(timeout_us == 0 ? 1000000000ull : timeout_us * 1000ull);
+  return DIT_OK;
+}
+
+int dit_selftest_wait_timeout(unsigned long long timeout_us, void* stream) {
+  if (timeout_us == 0 || timeout_us > 10000000ull) return DIT_ERR_INVALID_ARG;
+  selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(timeout_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+const char* dit_status_str(int status) {
+  switch (status & 0xFF) {
+    case DIT_OK: return "DIT_OK";
+    case DIT_ERR_INVALID_ARG: return "DIT_ERR_INVALID_ARG";
+    case DIT_ERR_UNSUPPORTED: return "DIT_ERR_UNSUPPORTED";
+    case DIT_ERR_MISALIGNED: return "DIT_ERR_MISALIGNED";
+    case DIT_ERR_CUDA: return "DIT_ERR_CUDA";
+    case DIT_ERR_TIMEOUT: return "DIT_ERR_TIMEOUT";
+    default: return "DIT_ERR_UNKNOWN";
+  }
+}
+
+int dit_version(void) { return 100; }
+
+}  // extern "C"

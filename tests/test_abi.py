@@ -1,0 +1,128 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared symbol, and
+host-side validation rejects bad arguments before anything reaches CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dit_attn.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dit_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from long_sequence_attention_b200 import build
+    build.build()
+    import long_sequence_attention_b200 as lsa
+    return lsa
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("dit_attn_fwd", "dit_attn_fwd_chunk", "dit_attn_merge", "dit_quant_fp8",
+              "dit_quant_fp8_workspace_bytes", "dit_device_status", "dit_status_str", "dit_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for name in _declared():
+        assert hasattr(raw, name), name
+
+
+def test_only_dit_symbols_exported(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    syms = [l.split()[-1] for l in out.splitlines() if l.strip()]
+    assert syms and all(s.startswith("dit_") for s in syms), syms
+
+
+def test_status_strings_and_version(lib):
+    assert lib.status_str(0) == "DIT_OK"
+    assert lib.status_str(5) == "DIT_ERR_TIMEOUT"
+    assert lib.status_str(5 | (3 << 8)) == "DIT_ERR_TIMEOUT"
+    assert lib.dit_version() >= 100
+
+
+# Fake, 256-byte aligned, non-null "device" addresses: validation must reject the call
+# before touching them.  Every call below has at least one invalid argument, so nothing is
+# ever launched on these addresses (not even on a machine with a GPU).
+A = 1 << 40
+Bp = A + (1 << 30)
+Cp = A + (2 << 30)
+O = A + (3 << 30)
+L = A + (4 << 30)
+
+
+def _chunk(lib, **kw):
+    args = dict(q=A, k=Bp, v=Cp, out=O, lse=L, B=1, H=2, S_q=256, S_kv=256, D=64, k0=0, k1=256,
+                scale=0.125, dtype=0, out_dtype=2, descale=None, stream=None)
+    args.update(kw)
+    return lib.lib.dit_attn_fwd_chunk(args["q"], args["k"], args["v"], args["out"], args["lse"], args["B"],
+                                      args["H"], args["S_q"], args["S_kv"], args["D"], args["k0"], args["k1"],
+                                      args["scale"], args["dtype"], args["out_dtype"], args["descale"],
+                                      args["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(out=None), 1), (dict(B=0), 1), (dict(H=0), 1), (dict(S_q=0), 1),
+    (dict(S_kv=0), 1), (dict(k0=-1), 1), (dict(k0=10, k1=5), 1), (dict(k1=257), 1),
+    (dict(scale=0.0), 1), (dict(scale=-1.0), 1), (dict(scale=float("inf")), 1), (dict(scale=float("nan")), 1),
+    (dict(dtype=7), 1), (dict(out_dtype=1), 1), (dict(D=96), 2), (dict(D=256), 2),
+    (dict(dtype=1, D=64, descale=A + 64), 2), (dict(dtype=1, D=128, descale=None), 1),
+    (dict(q=A + 8), 3), (dict(out=O + 4), 3), (dict(lse=L + 2), 3),
+    (dict(out=A + 128), 1),            # output overlaps q
+    (dict(lse=O + 64), 1),             # lse overlaps out
+])
+def test_chunk_validation(lib, kw, code):
+    assert _chunk(lib, **kw) == code
+
+
+def test_fwd_validation(lib):
+    f = lib.lib.dit_attn_fwd
+    assert f(None, Bp, Cp, O, L, 1, 2, 256, 64, 0.125, 0, None, None) == 1
+    assert f(A, Bp, Cp, O, L, 1, 2, 256, 80, 0.125, 0, None, None) == 2
+
+
+def test_merge_validation(lib):
+    vp = ctypes.c_void_p
+    outs = (vp * 2)(Bp, Cp)
+    lses = (vp * 2)(L, L + 4096)
+    m = lib.lib.dit_attn_merge
+    assert m(outs, lses, 0, O, None, 1, 2, 8, 64, 2, 0, None) == 1          # n_chunks
+    assert m(outs, lses, 17, O, None, 1, 2, 8, 64, 2, 0, None) == 1
+    assert m(outs, lses, 2, O, None, 1, 2, 8, 96, 2, 0, None) == 2          # D
+    assert m(outs, lses, 2, O, None, 1, 2, 8, 64, 1, 0, None) == 1          # in dtype
+    assert m(outs, lses, 2, O + 8, None, 1, 2, 8, 64, 2, 0, None) == 3      # misaligned out
+    bad = (vp * 2)(Bp + 4, Cp)
+    assert m(bad, lses, 2, O, None, 1, 2, 8, 64, 2, 0, None) == 3
+    alias = (vp * 2)(O, Cp)
+    assert m(alias, lses, 2, O, None, 1, 2, 8, 64, 2, 0, None) == 1         # out aliases a partial
+    null = (vp * 2)(Bp, None)
+    assert m(null, lses, 2, O, None, 1, 2, 8, 64, 2, 0, None) == 1
+
+
+def test_quant_validation(lib):
+    q = lib.lib.dit_quant_fp8
+    ws = lib.dit_quant_fp8_workspace_bytes(1 << 20)
+    assert ws == 4 * 128
+    assert lib.dit_quant_fp8_workspace_bytes(1) == 4
+    assert lib.dit_quant_fp8_workspace_bytes(1 << 40) == 4 * 1184
+    assert q(None, Bp, L, 1 << 20, Cp, ws, None) == 1
+    assert q(A, Bp, L, 0, Cp, ws, None) == 1
+    assert q(A, Bp, L, 1 << 20, Cp, ws - 4, None) == 1                       # workspace too small
+    assert q(A + 2, Bp, L, 1 << 20, Cp, ws, None) == 3
+    assert q(A, A + 64, L, 1 << 20, Cp, ws, None) == 1                       # output overlaps input
+
+
+def test_selftest_validation(lib):
+    assert lib.lib.dit_selftest_wait_timeout(0, None) == 1
+    assert lib.lib.dit_selftest_wait_timeout(10 ** 9, None) == 1
