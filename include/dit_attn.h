@@ -119,6 +119,30 @@ int dit_quant_fp8(const void* x_bf16, void* x_fp8, float* descale, long long n, 
                   size_t workspace_bytes, void* stream);
 
 /*
+ * dit_quant_fp8_noalloc - the same quantisation as dit_quant_fp8, for callers that cannot
+ * allocate device memory: code that runs where cudaMalloc is off limits (for example while
+ * a stream is being captured into a CUDA graph, or inside a framework whose allocator owns
+ * all device memory and forbids raw allocations), and so has no way to provide the
+ * workspace.  The pages have no counterpart to this call; it exists for such callers only.
+ *
+ *   x_bf16, x_fp8, descale, n: as for dit_quant_fp8; the caller still provides these.
+ *   Scratch: a 4736-byte array of partial maxima (1184 floats) that lives in the library's
+ *   own device data, so every GPU that loads the library keeps it until the process exits.
+ *   The call allocates and frees nothing.  Every n >= 1 fits: the first pass uses at most
+ *   1184 blocks, one scratch slot each; a block count above the array's size would be
+ *   rejected with DIT_ERR_UNSUPPORTED.
+ *   Set-up: the first call on each device (with that device current) looks up the array's
+ *   device address with cudaGetSymbolAddress; make that first call before any stream
+ *   capture.  Later calls reuse the address.
+ *   Sharing: all calls on a device share the one array and it keeps the last call's
+ *   contents.  Nothing in it needs to start at zero (each call writes every slot it reads
+ *   before reading it), but calls whose kernels overlap on the GPU (different streams, no
+ *   ordering between them) race on the array and give wrong results; order them.
+ */
+int dit_quant_fp8_noalloc(const void* x_bf16, void* x_fp8, float* descale, long long n,
+                          void* stream);
+
+/*
  * dit_device_status - synchronises the current device, then reads the device status word
  * into *status: DIT_OK, or DIT_ERR_TIMEOUT | (site << 8) when a bounded wait inside a
  * kernel ran out (the kernel then wound down without hanging; its outputs are invalid).

@@ -1,7 +1,7 @@
 """Python binding of the DiT joint-attention library for B200 (sm_100a).
 
 Argument marshalling only: every computation runs in the CUDA kernels of
-``libdit_attn.so`` (built in-tree by ``long_sequence_attention_b200.build``).  The C
+``libdit_attn.so`` (built in-tree by ``long_sequence_attention_b200/build.py``).  The C
 functions keep their names here (``dit_attn_fwd``, ``dit_attn_fwd_chunk``,
 ``dit_attn_merge``, ``dit_quant_fp8`` ...); tensors may be passed as torch CUDA tensors or
 as raw device addresses (ints).  A non-zero status raises ``DitError``.
@@ -34,7 +34,7 @@ class DitError(RuntimeError):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m long_sequence_attention_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python long_sequence_attention_b200/build.py` "
                           "(nvcc, sm_100a). There is no CPU fallback.")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, f, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong
@@ -45,6 +45,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_quant_fp8_workspace_bytes.argtypes = [ll]
     lib.dit_quant_fp8_workspace_bytes.restype = sz
     lib.dit_quant_fp8.argtypes = [vp, vp, vp, ll, vp, sz, vp]
+    lib.dit_quant_fp8_noalloc.argtypes = [vp, vp, vp, ll, vp]
+    lib.dit_quant_fp8_noalloc.restype = ctypes.c_int
     lib.dit_device_status.argtypes = [ctypes.POINTER(i), i]
     lib.dit_set_wait_timeout_us.argtypes = [ull]
     lib.dit_selftest_wait_timeout.argtypes = [ull, vp]
@@ -118,6 +120,13 @@ def dit_quant_fp8_workspace_bytes(n: int) -> int:
 def dit_quant_fp8(x_bf16, x_fp8, descale, n: int, workspace, workspace_bytes: int, stream=None) -> None:
     _check(lib.dit_quant_fp8(_ptr(x_bf16), _ptr(x_fp8), _ptr(descale), int(n), _ptr(workspace),
                              int(workspace_bytes), _stream(stream)), "dit_quant_fp8")
+
+
+def dit_quant_fp8_noalloc(x_bf16, x_fp8, descale, n: int, stream=None) -> None:
+    """dit_quant_fp8 without a workspace, for callers that cannot allocate device memory
+    (the scratch is a small array inside the library's device data; see the header)."""
+    _check(lib.dit_quant_fp8_noalloc(_ptr(x_bf16), _ptr(x_fp8), _ptr(descale), int(n), _stream(stream)),
+           "dit_quant_fp8_noalloc")
 
 
 def dit_device_status(clear: bool = True) -> int:

@@ -115,6 +115,40 @@ __global__ void selftest_wait_kernel(unsigned long long timeout_ns) {
 
 }  // namespace
 
+// ---------------------------------------------------------------------------------------
+// Scratch of dit_quant_fp8_noalloc: one partial absolute maximum per block of the first
+// quantisation pass.  It is part of the loaded module, so every GPU that loads this library
+// holds these 4736 bytes until the process exits; no call allocates anything.  Host code must
+// not hand this name to a kernel (on the host it is only a stand-in for the symbol): the
+// device address is looked up once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------------------
+constexpr int kNoAllocScratchFloats = dit::kQuantMaxBlocks;
+static __device__ __align__(256) float g_quant_noalloc_scratch[kNoAllocScratchFloats];
+static_assert(dit::kQuantMaxBlocks <= kNoAllocScratchFloats, "scratch must hold every partial maximum");
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+float* g_noalloc_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the static scratch on the current device (set-up on first use per device).
+int noalloc_scratch(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return DIT_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_scratch_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_quant_noalloc_scratch) != cudaSuccess || p == nullptr) return DIT_ERR_CUDA;
+    g_noalloc_scratch_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_scratch_ptr[dev];
+  return DIT_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
@@ -229,6 +263,26 @@ int dit_quant_fp8(const void* x_bf16, void* x_fp8, float* descale, long long n, 
   absmax_partial_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, partials);
   if (cudaGetLastError() != cudaSuccess) return DIT_ERR_CUDA;
   quant_e4m3_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, partials, g,
+                                                  static_cast<uint8_t*>(x_fp8), descale);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
+}
+
+int dit_quant_fp8_noalloc(const void* x_bf16, void* x_fp8, float* descale, long long n, void* stream) {
+  if (x_bf16 == nullptr || x_fp8 == nullptr || descale == nullptr) return DIT_ERR_INVALID_ARG;
+  if (n < 1) return DIT_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(x_fp8, 16) || !aligned(descale, 4)) return DIT_ERR_MISALIGNED;
+  if (overlaps(x_fp8, n, x_bf16, n * 2) || overlaps(descale, 4, x_bf16, n * 2) || overlaps(descale, 4, x_fp8, n))
+    return DIT_ERR_INVALID_ARG;
+  const int g = quant_blocks(n);
+  if (g > kNoAllocScratchFloats) return DIT_ERR_UNSUPPORTED;  // more partials than the static scratch holds
+  float* scratch = nullptr;
+  const int rc = noalloc_scratch(&scratch);
+  if (rc != DIT_OK) return rc;
+  // Pass 1 writes every slot 0..g-1 before pass 2 reads them, so nothing needs clearing.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  absmax_partial_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, scratch);
+  if (cudaGetLastError() != cudaSuccess) return DIT_ERR_CUDA;
+  quant_e4m3_kernel<<<g, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x_bf16), n, scratch, g,
                                                   static_cast<uint8_t*>(x_fp8), descale);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
