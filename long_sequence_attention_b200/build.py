@@ -1,6 +1,8 @@
 """Build the CUDA library in-tree: long_sequence_attention_b200/libdit_attn.so (sm_100a).
 
-    python -m long_sequence_attention_b200.build [--force] [--verbose]
+    python long_sequence_attention_b200/build.py [--force] [--verbose]
+
+(run it by path: importing the package first would load the library it is about to replace)
 
 One translation unit (csrc/dit_attn.cu includes every kernel), compiled by nvcc with
 -gencode arch=compute_100a,code=sm_100a.  The runtime is linked statically and the driver's

@@ -19,8 +19,8 @@ def _declared():
 
 @pytest.fixture(scope="module")
 def lib():
-    from long_sequence_attention_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import long_sequence_attention_b200 as lsa
     return lsa
 
