@@ -13,11 +13,17 @@
 // Work unit: one CTA per (b, h, 256 query rows) = two 128-row Q tiles that ping-pong, so the
 // exponentials of one tile overlap the tensor-core work of the other.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    MMA issuer (one thread issues every tcgen05.mma and commit)
 //   warp  9    TMA producer (Q once, then a ring of K stages and a ring of V stages)
+//   warps 10-11 idle (they complete the third warpgroup)
+// The block launches with 168 registers per thread; the third warpgroup then gives
+// registers back (setmaxnreg.dec to kRegsCtl) and the softmax warpgroups take them
+// (setmaxnreg.inc to kRegsSoftmax): 2*128*216 + 128*72 = 64512 = 384*168, so the increase
+// never waits on registers that do not exist.  The host checks the compiled register count
+// against that sum before the first launch.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).  P (bf16 or
 // e4m3) is written over the first columns of S and read from TMEM by the P.V MMA.
@@ -69,6 +75,23 @@ __device__ __forceinline__ float exp2_fma(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
+// The same evaluation for two values at once with packed fp32x2 instructions.
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x, magic);
+  const uint64_t f = f2_sub(x, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(0.0551716685295105f, 0.0551716685295105f), f,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  p = f2_fma(p, f, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  p = f2_fma(p, f, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  e0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  e1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 template <int D, bool FP8>
 struct AttnCfg {
   static constexpr int kBM = 128;                       // query rows per tile
@@ -84,7 +107,11 @@ struct AttnCfg {
   static constexpr int kUmmaK = 32 / kElem;             // K per MMA instruction (32 bytes)
   static constexpr int kQKSteps = kRowBytes / 32;       // MMAs per S tile
   static constexpr int kPVSteps = kBN / kUmmaK;         // MMAs per P.V
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 384;
+  static constexpr int kRegsLaunch = 168;      // per thread at launch (__launch_bounds__(384, 1))
+  static constexpr int kRegsSoftmax = 216;     // softmax warpgroups after setmaxnreg.inc
+  static constexpr int kRegsCtl = 72;          // MMA / TMA warpgroup after setmaxnreg.dec
+  static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsCtl <= kThreads * kRegsLaunch, "register split");
   static constexpr int kMmaWarp = 8;
   static constexpr int kTmaWarp = 9;
   static constexpr int kTmemCols = 512;
@@ -93,6 +120,12 @@ struct AttnCfg {
   // most probabilities are normal numbers rather than subnormals.
   static constexpr float kRescaleLog2 = FP8 ? 4.0f : 8.0f;
   static constexpr float kPShift = FP8 ? 4.0f : 0.0f;
+  // exp2 split: of every 8 column pairs, this many use the FMA-pipe polynomial
+#ifdef DIT_EMU_PER8
+  static constexpr int kEmuPer8 = DIT_EMU_PER8;
+#else
+  static constexpr int kEmuPer8 = 2;
+#endif
 
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
@@ -108,7 +141,7 @@ struct AttnCfg {
 };
 
 template <int D, bool FP8>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   using C = AttnCfg<D, FP8>;
@@ -161,6 +194,8 @@ __global__ void __launch_bounds__(320, 1)
   uint8_t* sK = smem + C::kOffK;
   uint8_t* sV = smem + C::kOffV;
 
+  if (warp >= 8) {
+    regs_dec<C::kRegsCtl>();
   if (warp == C::kTmaWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -212,23 +247,28 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t fmt = FP8 ? 0u : 1u;
       constexpr uint32_t id_s = instr_desc(fmt, false, 128, C::kBN);
       constexpr uint32_t id_o = instr_desc(fmt, true, 128, D);
-      const uint32_t q_addr = smem_u32(sQ), k_addr = smem_u32(sK), v_addr = smem_u32(sV);
 
+      // Descriptors differ only in their start-address field (bits 0..13 of the low word,
+      // address >> 4; shared-memory addresses stay below 2^18), so every K step is the low
+      // word of a base descriptor plus (offset >> 4), with one high word for all of them.
+      const uint64_t dq = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(sV), C::kBlkBytes, 1024);
+      const uint32_t qk_hi = static_cast<uint32_t>(dq >> 32), v_hi = static_cast<uint32_t>(dv >> 32);
+      const uint32_t q_lo = static_cast<uint32_t>(dq), k_lo = static_cast<uint32_t>(dk),
+                     v_lo = static_cast<uint32_t>(dv);
       auto issue_s = [&](int t, int ks) {
-        const uint32_t a0 = q_addr + t * C::kTileBytes;
-        const uint32_t b0 = k_addr + ks * C::kTileBytes;
+        const uint32_t a0 = q_lo + ((t * C::kTileBytes) >> 4);
+        const uint32_t b0 = k_lo + ((ks * C::kTileBytes) >> 4);
         const uint32_t d = tmem_base + (t ? C::kColS1 : C::kColS0);
 #pragma unroll
         for (int kk = 0; kk < C::kQKSteps; ++kk) {
-          const uint32_t off = (kk * 32 / 128) * C::kBlkBytes + (kk * 32) % 128;
-          const uint64_t ad = smem_desc_sw128(a0 + off, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(b0 + off, 16, 1024);
-          if constexpr (FP8) mma_f8_ss(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
-          else mma_f16_ss(d, ad, bd, id_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk * 32 / 128) * C::kBlkBytes + (kk * 32) % 128) >> 4;
+          mma_ss_lohi(FP8, d, a0 + off, qk_hi, b0 + off, qk_hi, id_s, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
-        const uint32_t b0 = v_addr + vs * C::kTileBytes;
+        const uint32_t b0 = v_lo + ((vs * C::kTileBytes) >> 4);
         const uint32_t a_tm = tmem_base + (t ? C::kColS1 : C::kColS0);
         const uint32_t d = tmem_base + (t ? C::kColO1 : C::kColO0);
 #pragma unroll
@@ -236,10 +276,8 @@ __global__ void __launch_bounds__(320, 1)
           // V tile is [kv rows][D] with D contiguous: MN-major B operand.  One MMA covers
           // kUmmaK kv rows (groups of 8 rows 1024 bytes apart) and all of D (64-element,
           // 128-byte atoms kBlkBytes apart).
-          const uint64_t bd = smem_desc_sw128(b0 + kk * C::kUmmaK * 128, C::kBlkBytes, 1024);
-          const uint32_t acc_flag = (acc || kk > 0) ? 1u : 0u;
-          if constexpr (FP8) mma_f8_ts(d, a_tm + kk * 8, bd, id_o, acc_flag);
-          else mma_f16_ts(d, a_tm + kk * 8, bd, id_o, acc_flag);
+          const uint32_t off = (kk * C::kUmmaK * 128) >> 4;
+          mma_ts_lohi(FP8, d, a_tm + kk * 8, b0 + off, v_hi, id_o, (acc || kk > 0) ? 1u : 0u);
         }
       };
 
@@ -288,8 +326,10 @@ __global__ void __launch_bounds__(320, 1)
       tc_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, tmo);
     }
+  }  // warps 10 and 11 have no role
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
+    regs_inc<C::kRegsSoftmax>();
     const int t = warp >> 2;                // Q tile of this warpgroup
     const int quad = warp & 3;              // TMEM lane quadrant of this warp
     const int row = quad * 32 + lane;       // row within the tile == TMEM lane
@@ -317,13 +357,19 @@ __global__ void __launch_bounds__(320, 1)
         for (int c = 0; c < 128; ++c)
           if (c >= valid) s[c] = 0xFF800000u;                  // -inf
       }
+      // row max of the tile: 8 independent chains of 3-input max
       float mx[8];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) mx[c] = __uint_as_float(s[c]);
+      for (int i = 0; i < 8; ++i)
+        mx[i] = fmax3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], __uint_as_float(s[c]));
-      const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      for (int c = 24; c < 120; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          mx[i] = fmax3(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __uint_as_float(s[120 + i]));
+      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
       const float m_new = fmaxf(m_use, mt);
       const bool need = (m_new - m_use) * cl > C::kRescaleLog2;   // true on the first tile
       float alpha = 1.0f;
@@ -331,36 +377,51 @@ __global__ void __launch_bounds__(320, 1)
         alpha = ex2_approx((m_use - m_new) * cl);              // 0 when m_use = -inf
         m_use = m_new;
       }
+      // p = 2^(cl*s - mc), two lanes per instruction; pairs (c2 & 7) < kEmuPer8 go to the
+      // FMA-pipe polynomial, the rest to the MUFU ex2
       const float mc = m_use * cl - C::kPShift;
-      float sum[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pa[32], pb[32];               // P words for TMEM columns [0,32) and [32,64)
-      if constexpr (!FP8) {
+      const uint64_t cl2 = f2_pack(cl, cl), nmc2 = f2_pack(-mc, -mc);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+      // Two halves of 32 column pairs; each half's P words go to TMEM as soon as they are
+      // complete, so their registers (and the scores they came from) are free for the rest.
 #pragma unroll
-        for (int c2 = 0; c2 < 64; ++c2) {
-          const float x0 = fmaf(__uint_as_float(s[2 * c2]), cl, -mc);
-          const float x1 = fmaf(__uint_as_float(s[2 * c2 + 1]), cl, -mc);
-          float e0, e1;
-          if ((c2 & 3) == 3) { e0 = exp2_fma(x0); e1 = exp2_fma(x1); }
-          else { e0 = ex2_approx(x0); e1 = ex2_approx(x1); }
-          sum[c2 & 3] += e0 + e1;
-          if (c2 < 32) pa[c2] = pack_bf16x2(e0, e1);
-          else pb[c2 - 32] = pack_bf16x2(e0, e1);
-        }
-        tmem_st32(tS, pa);
-        tmem_st32(tS + 32, pb);
-      } else {
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pw[32];
 #pragma unroll
-        for (int c4 = 0; c4 < 32; ++c4) {
-          float e[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float x = fmaf(__uint_as_float(s[4 * c4 + u]), cl, -mc);
-            e[u] = ((c4 & 3) == 3) ? exp2_fma(x) : ex2_approx(x);
+        for (int i = 0; i < 32; ++i) {
+          const int c2 = half * 32 + i;
+          const uint64_t x =
+              f2_fma(f2_pack(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), cl2, nmc2);
+          float x0, x1, e0, e1;
+          f2_unpack(x, x0, x1);
+          if ((c2 & 7) < C::kEmuPer8) {
+            exp2_fma2(x0, x1, e0, e1);
+          } else {
+            e0 = ex2_approx(x0);
+            e1 = ex2_approx(x1);
           }
-          sum[c4 & 3] += (e[0] + e[1]) + (e[2] + e[3]);
-          pa[c4] = pack_e4m3x4(e[0], e[1], e[2], e[3]);
+          acc[c2 & 3] = f2_add(acc[c2 & 3], f2_pack(e0, e1));
+          if constexpr (!FP8) {
+            pw[i] = pack_bf16x2(e0, e1);
+          } else {
+            // four e4m3 per TMEM column: pair 2q in bytes 0-1, pair 2q+1 in bytes 2-3
+            const uint32_t h = pack_e4m3x2(e0, e1);
+            if (i & 1) pw[i >> 1] |= h << 16;
+            else pw[i >> 1] = h;
+          }
         }
-        tmem_st32(tS, pa);
+        if constexpr (!FP8) {
+          tmem_st32(tS + 32 * half, pw);
+        } else {
+          tmem_st16(tS + 16 * half, *reinterpret_cast<uint32_t(*)[16]>(pw));
+        }
+      }
+      float sum;
+      {
+        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
+        float lo, hi;
+        f2_unpack(f2_add(a01, a23), lo, hi);
+        sum = lo + hi;
       }
       tmem_st_wait();
       // O_t is quiescent here (PV_t(j-1) completed before S_t(j) was signalled).
@@ -375,7 +436,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         tmem_st_wait();
       }
-      l = fmaf(l, alpha, (sum[0] + sum[1]) + (sum[2] + sum[3]));
+      l = fmaf(l, alpha, sum);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p_full + t);

@@ -78,11 +78,32 @@ int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
   return DIT_OK;
 }
 
+// The forward kernel re-splits registers between warpgroups with setmaxnreg; the increase
+// only completes if the block was launched with at least the registers the split adds up to.
+// Refuse to launch a build where that does not hold (it would wait forever).
+template <int D, bool FP8>
+int check_register_split() {
+  using C = AttnCfg<D, FP8>;
+  static std::atomic<int> verdict{0};   // 0 unknown, 1 ok, 2 bad
+  int v = verdict.load();
+  if (v == 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8>) != cudaSuccess) return DIT_ERR_CUDA;
+    const long long launched = static_cast<long long>(attr.numRegs) * C::kThreads;
+    const long long wanted = 2LL * 128 * C::kRegsSoftmax + 128LL * C::kRegsCtl;
+    v = (attr.numRegs == C::kRegsLaunch && launched >= wanted) ? 1 : 2;
+    verdict.store(v);
+  }
+  return v == 1 ? DIT_OK : DIT_ERR_UNSUPPORTED;
+}
+
 template <int D, bool FP8>
 int launch_attn(const void* q, const void* k, const void* v, const AttnParams& prm, cudaStream_t st) {
   using C = AttnCfg<D, FP8>;
   static std::atomic<uint64_t> attr_done{0};
-  int rc = ensure_smem_attr(attn_fwd_kernel<D, FP8>, C::kSmemBytes, attr_done);
+  int rc = check_register_split<D, FP8>();
+  if (rc != DIT_OK) return rc;
+  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8>, C::kSmemBytes, attr_done);
   if (rc != DIT_OK) return rc;
   CUtensorMap tq, tk, tv;
   const int BH = prm.B * prm.H;

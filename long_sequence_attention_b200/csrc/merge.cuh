@@ -57,27 +57,40 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const MergeParams p) {
        u += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long row = u / tpr;
     const int col = static_cast<int>(u - row * tpr) * 8;
+    const long long e = row * p.D + col;
     float M = -INFINITY;
     for (int c = 0; c < p.n; ++c) M = fmaxf(M, __ldg(p.lses[c] + row));
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     float L = 0.0f;
     if (M != -INFINITY) {
-      for (int c = 0; c < p.n; ++c) {
-        const float lc = __ldg(p.lses[c] + row);
-        const float w = __expf(lc - M);                       // exactly 0 for an empty chunk
-        L += w;
-        if (w != 0.0f) {
-          float v[8];
-          load8(p.outs[c], row * p.D + col, p.in_fp32 != 0, v);
+      // Four chunks at a time: all their loads are issued before any is used, so each thread
+      // keeps up to 4 x 32 bytes in flight.  An empty chunk (lse = -inf) has weight exactly 0
+      // and its values are discarded by a select, whatever its buffer holds.
+      for (int c0 = 0; c0 < p.n; c0 += 4) {
+        float v[4][8];
+        float w[4];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, v[i], acc[i]);
+        for (int k = 0; k < 4; ++k) {
+          const int c = c0 + k;
+          w[k] = 0.0f;
+          if (c < p.n) {
+            w[k] = __expf(__ldg(p.lses[c] + row) - M);
+            load8(p.outs[c], e, p.in_fp32 != 0, v[k]);
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          if (c0 + k < p.n) {
+            L += w[k];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = (w[k] != 0.0f) ? fmaf(w[k], v[k][i], acc[i]) : acc[i];
+          }
         }
       }
       const float inv = 1.0f / L;
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] *= inv;
     }
-    const long long e = row * p.D + col;
     if (p.out_fp32) {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + e);
       dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);

@@ -57,6 +57,26 @@ def test_merge_of_empty_and_full_chunk_is_identity(cuda_lib):
     assert torch.equal(mo, o) and torch.allclose(ml, l, atol=1e-6, rtol=0)
 
 
+@pytest.mark.parametrize("n", [2, 5])
+def test_merge_ignores_garbage_in_empty_chunks(cuda_lib, n):
+    """An empty chunk (lse = -inf) has weight 0: whatever its out buffer holds (NaN, inf)
+    must not reach the result."""
+    import torch
+    B, H, S, D = 1, 2, 130, 128
+    good_o, _ = normal_bf16((B, H, S, D), 77)
+    good_l = np.random.default_rng(1).normal(size=(B, H, S)).astype(np.float32)
+    outs_h = [good_o] + [np.full((B, H, S, D), np.nan, dtype=np.float32) for _ in range(n - 1)]
+    outs_h[-1][..., ::2] = np.inf
+    lses_h = [good_l] + [np.full((B, H, S), -np.inf, dtype=np.float32) for _ in range(n - 1)]
+    outs = [torch.from_numpy(o).cuda() for o in outs_h]
+    lses = [torch.from_numpy(l).cuda() for l in lses_h]
+    mo, ml = cuda_lib.merge(outs, lses, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.isfinite(mo).all()
+    assert torch.equal(mo.cpu(), torch.from_numpy(good_o))
+    assert torch.allclose(ml.cpu(), torch.from_numpy(good_l), atol=1e-6, rtol=0)
+
+
 # ------------------------------------------------------------------------------ E4M3 quantiser
 def _quant_dev(lsa, x_bits):
     import torch
