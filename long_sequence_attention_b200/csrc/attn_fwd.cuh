@@ -10,8 +10,12 @@
 // section 3.2.2): a ring step attends the local queries to one block of keys and the partial
 // results are combined afterwards by the log-sum-exp merge (merge.cuh).
 //
-// Work unit: one CTA per (b, h, 256 query rows) = two 128-row Q tiles that ping-pong, so the
-// exponentials of one tile overlap the tensor-core work of the other.
+// Work unit: (b, h, 256 query rows) = two 128-row Q tiles that ping-pong, so the
+// exponentials of one tile overlap the tensor-core work of the other.  The kernel is
+// persistent: a grid of at most one CTA per SM walks the units u = blockIdx.x + k*gridDim.x
+// (query block fastest, so the CTAs running at the same time share a head's K/V in L2).
+// Barrier phases and ring stages follow a per-CTA running tile count g = it * n_kv + j, so
+// the next unit's Q load, its first S MMAs and this unit's epilogue overlap.
 //
 // Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
@@ -49,6 +53,8 @@ namespace dit {
 
 struct AttnParams {
   int B, H, S_q, S_kv;
+  int n_qblk;              // ceil(S_q / 256) query blocks per head
+  int n_units;             // n_qblk * H * B
   int k0, k1;
   float scale;             // softmax scale applied to q.k
   const float* descale;    // e4m3 path: device pointer to {descale_q, descale_k, descale_v}
@@ -132,7 +138,7 @@ struct AttnCfg {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -158,14 +164,16 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_p_full = bar_s_full + 2;              // [2]
   uint64_t* bar_o_final = bar_p_full + 2;             // [2]
   uint64_t* bar_drain = bar_o_final + 2;              // [1]
+  uint64_t* bar_q_empty = bar_drain + 1;              // [1]
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int bh = blockIdx.z * p.H + blockIdx.y;
-  const int q_start = blockIdx.x * (2 * C::kBM);
   const int n_kv = (p.k1 - p.k0 + C::kBN - 1) / C::kBN;   // >= 1 (empty ranges never launch)
+  // unit -> (head index b*H + h, first query row); query block fastest
+  auto unit_bh = [&](int u) { return u / p.n_qblk; };
+  auto unit_q0 = [&](int u) { return (u % p.n_qblk) * (2 * C::kBM); };
   const uint64_t tmo = p.timeout_ns;
 
   if (threadIdx.x == C::kTmaWarp * 32) {
@@ -178,6 +186,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(bar_o_final + t, 1);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_q_empty, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -202,36 +211,44 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int b = 0; b < C::kNBlk; ++b)
-          tma_load_3d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
-                      q_start + t * C::kBM, bh);
-      int k_issued = 0, v_issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int kv_row = p.k0 + j * C::kBN;
-        const int ks = j % C::kKStages;
-        if (j >= C::kKStages &&
-            !mbar_wait(bar_k_empty + ks, ((j / C::kKStages) + 1) & 1, abort_flag, tmo, 1))
-          break;
-        mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
-        for (int b = 0; b < C::kNBlk; ++b)
-          tma_load_3d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
-                      b * C::kBoxInner, kv_row, bh);
-        k_issued = j + 1;
-        const int vs = j % C::kVStages;
-        if (j >= C::kVStages &&
-            !mbar_wait(bar_v_empty + vs, ((j / C::kVStages) + 1) & 1, abort_flag, tmo, 2))
-          break;
-        mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
-        for (int b = 0; b < C::kNBlk; ++b)
-          tma_load_3d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
-                      b * C::kBoxInner, kv_row, bh);
-        v_issued = j + 1;
+      int k_issued = 0, v_issued = 0, q_issued = 0;   // running counts over all units
+      bool ok = true;
+      for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+        const int bh = unit_bh(u), q0 = unit_q0(u);
+        // Q of this unit may overwrite the previous unit's only after its last S MMA.
+        if (it > 0 && !(ok = mbar_wait(bar_q_empty, (it - 1) & 1, abort_flag, tmo, 0))) break;
+        mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int b = 0; b < C::kNBlk; ++b)
+            tma_load_3d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
+                        q0 + t * C::kBM, bh);
+        q_issued = it + 1;
+        for (int j = 0; j < n_kv; ++j) {
+          const int g = it * n_kv + j;
+          const int kv_row = p.k0 + j * C::kBN;
+          const int ks = g % C::kKStages;
+          if (g >= C::kKStages &&
+              !(ok = mbar_wait(bar_k_empty + ks, ((g / C::kKStages) + 1) & 1, abort_flag, tmo, 1)))
+            break;
+          mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
+          for (int b = 0; b < C::kNBlk; ++b)
+            tma_load_3d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
+                        b * C::kBoxInner, kv_row, bh);
+          k_issued = g + 1;
+          const int vs = g % C::kVStages;
+          if (g >= C::kVStages &&
+              !(ok = mbar_wait(bar_v_empty + vs, ((g / C::kVStages) + 1) & 1, abort_flag, tmo, 2)))
+            break;
+          mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
+          for (int b = 0; b < C::kNBlk; ++b)
+            tma_load_3d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
+                        b * C::kBoxInner, kv_row, bh);
+          v_issued = g + 1;
+        }
       }
       // Drain: the last load armed on every stage must land before the CTA may exit
       // (a no-op in a healthy run, where the consumers already waited for all of them).
-      mbar_wait_drain(bar_q_full, 0, tmo);
+      if (q_issued > 0) mbar_wait_drain(bar_q_full, (q_issued - 1) & 1, tmo);
       for (int s = 0; s < C::kKStages; ++s) {
         const int last = s + ((k_issued - 1 - s) / C::kKStages) * C::kKStages;
         if (k_issued > s) mbar_wait_drain(bar_k_full + s, (last / C::kKStages) & 1, tmo);
@@ -281,45 +298,51 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
 
-      bool ok = mbar_wait(bar_q_full, 0, abort_flag, tmo, 3);
-      if (ok) tc_fence_after();
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int ks = j % C::kKStages;
-        if (!(ok = mbar_wait(bar_k_full + ks, (j / C::kKStages) & 1, abort_flag, tmo, 4))) break;
+      bool ok = true;
+      for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+        if (!(ok = mbar_wait(bar_q_full, it & 1, abort_flag, tmo, 3))) break;
         tc_fence_after();
-        const int jp = j - 1, vs = (j - 1) % C::kVStages;
-        if (j > 0) {
-          if (!(ok = mbar_wait(bar_v_full + vs, (jp / C::kVStages) & 1, abort_flag, tmo, 5))) break;
-          if (!(ok = mbar_wait(bar_p_full + 0, jp & 1, abort_flag, tmo, 6))) break;
+        const int g0 = it * n_kv;
+        for (int j = 0; ok && j < n_kv; ++j) {
+          const int g = g0 + j;
+          const int ks = g % C::kKStages;
+          if (!(ok = mbar_wait(bar_k_full + ks, (g / C::kKStages) & 1, abort_flag, tmo, 4))) break;
           tc_fence_after();
-          issue_pv(0, vs, jp > 0);
+          const int gp = g - 1, vs = (g - 1) % C::kVStages;
+          if (j > 0) {
+            if (!(ok = mbar_wait(bar_v_full + vs, (gp / C::kVStages) & 1, abort_flag, tmo, 5))) break;
+            if (!(ok = mbar_wait(bar_p_full + 0, gp & 1, abort_flag, tmo, 6))) break;
+            tc_fence_after();
+            issue_pv(0, vs, j - 1 > 0);
+          }
+          issue_s(0, ks);
+          tc_commit(bar_s_full + 0);
+          if (j > 0) {
+            if (!(ok = mbar_wait(bar_p_full + 1, gp & 1, abort_flag, tmo, 7))) break;
+            tc_fence_after();
+            issue_pv(1, vs, j - 1 > 0);
+            tc_commit(bar_v_empty + vs);
+          }
+          issue_s(1, ks);
+          tc_commit(bar_s_full + 1);
+          tc_commit(bar_k_empty + ks);
         }
-        issue_s(0, ks);
-        tc_commit(bar_s_full + 0);
-        if (j > 0) {
-          if (!(ok = mbar_wait(bar_p_full + 1, jp & 1, abort_flag, tmo, 7))) break;
-          tc_fence_after();
-          issue_pv(1, vs, jp > 0);
-          tc_commit(bar_v_empty + vs);
-        }
-        issue_s(1, ks);
-        tc_commit(bar_s_full + 1);
-        tc_commit(bar_k_empty + ks);
-      }
-      if (ok) {
-        const int jl = n_kv - 1, vs = jl % C::kVStages;
-        ok = mbar_wait(bar_v_full + vs, (jl / C::kVStages) & 1, abort_flag, tmo, 8);
-        if (ok) ok = mbar_wait(bar_p_full + 0, jl & 1, abort_flag, tmo, 9);
+        if (!ok) break;
+        tc_commit(bar_q_empty);                    // every S MMA of this unit is issued
+        const int gl = g0 + n_kv - 1, vs = gl % C::kVStages;
+        ok = mbar_wait(bar_v_full + vs, (gl / C::kVStages) & 1, abort_flag, tmo, 8);
+        if (ok) ok = mbar_wait(bar_p_full + 0, gl & 1, abort_flag, tmo, 9);
         if (ok) {
           tc_fence_after();
-          issue_pv(0, vs, jl > 0);
+          issue_pv(0, vs, n_kv > 1);
           tc_commit(bar_o_final + 0);
-          ok = mbar_wait(bar_p_full + 1, jl & 1, abort_flag, tmo, 10);
+          ok = mbar_wait(bar_p_full + 1, gl & 1, abort_flag, tmo, 10);
         }
         if (ok) {
           tc_fence_after();
-          issue_pv(1, vs, jl > 0);
+          issue_pv(1, vs, n_kv > 1);
           tc_commit(bar_o_final + 1);
+          tc_commit(bar_v_empty + vs);
         }
       }
       // Every MMA this thread issued must finish before TMEM is released.
@@ -341,12 +364,15 @@ __global__ void __launch_bounds__(384, 1)
     if constexpr (FP8) { dq = p.descale[0]; dk = p.descale[1]; dv = p.descale[2]; }
     const float scale_eff = p.scale * dq * dk;                 // natural-log units per raw score
     const float cl = scale_eff * 1.4426950408889634f;          // log2 units per raw score
-    float m_use = -INFINITY;                                   // running (lazy) max, raw units
-    float l = 0.0f;
     bool ok = true;
 
+    for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+    const int bh = unit_bh(u), q_start = unit_q0(u);
+    float m_use = -INFINITY;                                   // running (lazy) max, raw units
+    float l = 0.0f;
     for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + t, j & 1, abort_flag, tmo, 11 + t));
+      const int g = it * n_kv + j;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + t, g & 1, abort_flag, tmo, 11 + t));
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
@@ -443,7 +469,7 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // ---------------------------------------------------------------- epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final + t, 0, abort_flag, tmo, 13 + t));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final + t, it & 1, abort_flag, tmo, 13 + t));
     if (ok) {
       tc_fence_after();
       const int grow = q_start + t * C::kBM + row;
@@ -475,7 +501,10 @@ __global__ void __launch_bounds__(384, 1)
       if (store && p.lse != nullptr)
         p.lse[static_cast<size_t>(bh) * p.S_q + grow] =
             scale_eff * m_use + logf(l) - C::kPShift * 0.6931471805599453f;
+      // The O reads above end with tcgen05.wait::ld; the next unit's first P.V (which
+      // overwrites O_t) is issued only after this warpgroup publishes that unit's P_t.
     }
+    }  // units
   }
 
   tc_fence_before();

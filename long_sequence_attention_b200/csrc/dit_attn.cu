@@ -65,6 +65,22 @@ int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH) {
   return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
 }
 
+// Number of SMs of the current device (cached per device).
+int sm_count(int* out) {
+  static std::atomic<int> cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_CUDA;
+  if (dev >= 0 && dev < 64 && cache[dev].load() > 0) {
+    *out = cache[dev].load();
+    return DIT_OK;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return DIT_ERR_CUDA;
+  if (dev >= 0 && dev < 64) cache[dev].store(n);
+  *out = n;
+  return DIT_OK;
+}
+
 // Raise the dynamic shared-memory limit of a kernel once per device.
 template <typename K>
 int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
@@ -110,8 +126,13 @@ int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p
   if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH)) != DIT_OK) return rc;
   if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
   if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
-  const dim3 grid((prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM), prm.H, prm.B);
-  attn_fwd_kernel<D, FP8><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, prm);
+  AttnParams pr = prm;
+  pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
+  pr.n_units = pr.n_qblk * prm.H * prm.B;
+  int sms = 0;
+  if ((rc = sm_count(&sms)) != DIT_OK) return rc;
+  const int grid = pr.n_units < sms ? pr.n_units : sms;   // persistent: at most one CTA per SM
+  attn_fwd_kernel<D, FP8><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, pr);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 

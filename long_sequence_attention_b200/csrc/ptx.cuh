@@ -265,7 +265,20 @@ __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]
       : "memory");
 }
 
-// 128 consecutive columns in one go (four x32 loads, one wait).
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,"
+      "%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,"
+      "%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : DIT_O16(0), DIT_O16(16), DIT_O16(32), DIT_O16(48)
+      : "r"(taddr)
+      : "memory");
+}
+
+// 128 consecutive columns in one go (one x128 load, one wait).
 __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&r)[128]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x128.b32 "
@@ -341,6 +354,11 @@ __host__ __device__ constexpr uint32_t instr_desc(uint32_t ab_format, bool b_mn_
          | ((b_mn_major ? 1u : 0u) << 16)            // B major
          | ((static_cast<uint32_t>(N) >> 3) << 17)   // N / 8
          | ((static_cast<uint32_t>(M) >> 4) << 24);  // M / 16
+}
+
+// Named barrier among `count` threads (a multiple of 32); ids 1..15 (0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 // Warpgroup-wide register re-split (all 128 threads of the warpgroup execute it).
