@@ -51,6 +51,47 @@ def rank_info():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+def replica_seed_offset(rank: int) -> int:
+    """Each rank runs its own replica batch: the workload seeds shift by 10 per rank."""
+    return 10 * rank
+
+
+class Ranks:
+    """Process-group plumbing of a multi-rank run: every rank makes the same calls in the
+    same order; timing is reduced to the max over ranks.  With world == 1 it is a no-op."""
+
+    def __init__(self, world: int, backend: str = "nccl", device=None, timeout_s: int = 120):
+        self.world, self.backend, self.device, self.timeout_s = world, backend, device, timeout_s
+
+    def init(self):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            kw = {"device_id": self.device} if (self.backend == "nccl" and self.device is not None) else {}
+            dist.init_process_group(self.backend, timeout=datetime.timedelta(seconds=self.timeout_s), **kw)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.world == 1:
+            return float(x)
+        import torch
+        import torch.distributed as dist
+        dev = self.device if self.backend == "nccl" else "cpu"
+        t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -234,21 +275,14 @@ def run_ours(args, rank, local_rank, world):
 
     dev = torch.device(f"cuda:{local_rank}")
     torch.cuda.set_device(dev)
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    ranks = Ranks(world, "nccl", dev)
+    ranks.init()
     w = WORKLOADS[args.workload]
     fp8 = args.workload == "video"
-    data = make_qkv(w, seed_offset=rank * 10)          # each rank: its own replica batch
+    data = make_qkv(w, seed_offset=replica_seed_offset(rank))   # each rank: its own replica batch
     stream = torch.cuda.Stream(device=dev)
     step = Step(lsa, w, data, dev, fp8)
-
-    def barrier():
-        if world > 1:
-            import torch.distributed as dist
-            dist.barrier()
+    barrier = ranks.barrier
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -271,12 +305,7 @@ def run_ours(args, rank, local_rank, world):
         stream.synchronize()
     barrier()
     torch.cuda.synchronize()
-    elapsed_ms = t0.elapsed_time(t1)
-    if world > 1:
-        import torch.distributed as dist
-        tt = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = ranks.max(t0.elapsed_time(t1))
     status = lsa.dit_device_status(clear=True)
 
     full_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -286,12 +315,9 @@ def run_ours(args, rank, local_rank, world):
 
     # end to end through the C ABI with host buffers: pinned H2D of Q, K, V, the step, D2H of
     # the outputs, all inside the timed region
-    e2e = run_e2e(args, lsa, step, data, stream, dev)
+    e2e = run_e2e(args, lsa, step, data, stream, dev, ranks)
 
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
     if rank != 0:
         return
 
@@ -349,7 +375,7 @@ def run_ours(args, rank, local_rank, world):
     print(json.dumps(line), flush=True)
 
 
-def run_e2e(args, lsa, step, data, stream, dev):
+def run_e2e(args, lsa, step, data, stream, dev, ranks):
     import torch
     w = step.w
     host_in = [torch.from_numpy(data[n + "_bits"].view(np.int16)).view(torch.bfloat16).pin_memory() for n in "qkv"]
@@ -375,17 +401,18 @@ def run_e2e(args, lsa, step, data, stream, dev):
     with torch.cuda.stream(stream):
         one()
         stream.synchronize()
+        ranks.barrier()
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(n_steps):
             one()
         t1.record(stream)
     stream.synchronize()
-    ms = t0.elapsed_time(t1) / n_steps
+    ms = ranks.max(t0.elapsed_time(t1)) / n_steps
     bi = sum(h.numel() * h.element_size() for h in host_in)
     bo = sum(h.numel() * h.element_size() for h, _ in outs)
-    return {"value": round(step.flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(ms, 3),
-            "steps": n_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+    return {"value": round(step.flops * ranks.world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "steps": n_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
