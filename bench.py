@@ -342,8 +342,9 @@ def run_ours(args, rank, local_rank, world):
         "data": "synthetic (seeded N(0,1) rounded to bf16; no weights involved)",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "D": w.D, "scale": w.scale,
                    "n_chunks": w.n_chunks, "fp8_variant": fp8,
-                   "step": "dit_attn_fwd + %d x dit_attn_fwd_chunk + dit_attn_merge%s" % (
-                       len(step.bounds), " + 3 x dit_quant_fp8 + dit_attn_fwd(e4m3)" if fp8 else ""),
+                   "step": "dit_attn_fwd" + (" + %d x dit_attn_fwd_chunk + dit_attn_merge" % len(step.bounds)
+                                             if step.bounds else "")
+                           + (" + 3 x dit_quant_fp8 + dit_attn_fwd(e4m3)" if fp8 else ""),
                    "l2": "no flush: Q/K/V (%.0f MB) exceed the 126 MB L2" % (3 * w.B * w.H * w.S * w.D * 2 / 1e6),
                    "parallelism": "replicas%d" % world},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (dit_attn_fwd)",

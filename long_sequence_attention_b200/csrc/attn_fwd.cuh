@@ -126,12 +126,19 @@ struct AttnCfg {
   // most probabilities are normal numbers rather than subnormals.
   static constexpr float kRescaleLog2 = FP8 ? 4.0f : 8.0f;
   static constexpr float kPShift = FP8 ? 4.0f : 0.0f;
-  // exp2 split: of every 8 column pairs, this many use the FMA-pipe polynomial
+  static constexpr float kSumBound = 256.0f;           // = 2^(kRescaleLog2 + kPShift)
+  static constexpr int kPWordsHalf = FP8 ? 16 : 32;     // 32-bit P words per half row
+  // exp2 split: of every 8 column pairs, this many use the FMA-pipe polynomial (measured
+  // best: none at bf16 D=128, 1 at bf16 D=64, 2 for e4m3)
 #ifdef DIT_EMU_PER8
   static constexpr int kEmuPer8 = DIT_EMU_PER8;
 #else
-  static constexpr int kEmuPer8 = 2;
+  static constexpr int kEmuPer8 = FP8 ? 2 : (D == 64 ? 1 : 0);
 #endif
+  // bf16: exponentiate with the running max first and redo a tile exactly only when its row
+  // sum exceeds kSumBound.  e4m3 P is shifted up by 2^kPShift, so its sums sit near the bound
+  // and it always takes the max first.
+  static constexpr bool kSpeculative = !FP8;
 
   // shared memory layout (offsets from a 1024-byte aligned base)
   static constexpr int kOffQ = 0;
@@ -145,6 +152,63 @@ struct AttnCfg {
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(!FP8 || D == 128, "e4m3 path is built for D = 128");
 };
+
+// Columns c >= valid of a 128-column score row become -inf (keys past the range).
+__device__ __forceinline__ void mask_tail(uint32_t (&s)[128], int valid) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (c >= valid) s[c] = 0xFF800000u;
+}
+
+// Row max of 128 scores: 8 independent chains of 3-input max.
+__device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
+  float mx[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    mx[i] = fmax3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
+#pragma unroll
+  for (int c = 24; c < 120; c += 16)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      mx[i] = fmax3(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
+#pragma unroll
+  for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __uint_as_float(s[120 + i]));
+  return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+}
+
+// p = 2^(cl*s - mc) for the 128 scores of a row, two lanes per instruction; of every 8
+// column pairs, kEmu use the FMA-pipe polynomial and the rest the MUFU ex2.  Writes the P
+// words (bf16 pairs: 64 words, or e4m3 quads: 32 words) and the row sum.
+template <bool FP8, int kEmu>
+__device__ __forceinline__ void exp_pass(const uint32_t (&s)[128], float cl, float mc, uint32_t* pw, float& sum) {
+  const uint64_t cl2 = f2_pack(cl, cl), nmc2 = f2_pack(-mc, -mc);
+  uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int c2 = 0; c2 < 64; ++c2) {
+    const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), cl2, nmc2);
+    float x0, x1, e0, e1;
+    f2_unpack(x, x0, x1);
+    if ((c2 & 7) < kEmu) {
+      exp2_fma2(x0, x1, e0, e1);
+    } else {
+      e0 = ex2_approx(x0);
+      e1 = ex2_approx(x1);
+    }
+    acc[c2 & 3] = f2_add(acc[c2 & 3], f2_pack(e0, e1));
+    if constexpr (!FP8) {
+      pw[c2] = pack_bf16x2(e0, e1);
+    } else {
+      // four e4m3 per TMEM column: pair 2q in bytes 0-1, pair 2q+1 in bytes 2-3
+      const uint32_t h = pack_e4m3x2(e0, e1);
+      if (c2 & 1) pw[c2 >> 1] |= h << 16;
+      else pw[c2 >> 1] = h;
+    }
+  }
+  const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
+  float lo, hi;
+  f2_unpack(f2_add(a01, a23), lo, hi);
+  sum = lo + hi;
+}
 
 template <int D, bool FP8>
 __global__ void __launch_bounds__(384, 1)
@@ -378,77 +442,36 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
       const int valid = p.k1 - (p.k0 + j * C::kBN);
-      if (valid < C::kBN) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c >= valid) s[c] = 0xFF800000u;                  // -inf
-      }
-      // row max of the tile: 8 independent chains of 3-input max
-      float mx[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        mx[i] = fmax3(__uint_as_float(s[i]), __uint_as_float(s[i + 8]), __uint_as_float(s[i + 16]));
-#pragma unroll
-      for (int c = 24; c < 120; c += 16)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          mx[i] = fmax3(mx[i], __uint_as_float(s[c + i]), __uint_as_float(s[c + 8 + i]));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], __uint_as_float(s[120 + i]));
-      const float mt = fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
-      const float m_new = fmaxf(m_use, mt);
-      const bool need = (m_new - m_use) * cl > C::kRescaleLog2;   // true on the first tile
-      float alpha = 1.0f;
-      if (need) {
-        alpha = ex2_approx((m_use - m_new) * cl);              // 0 when m_use = -inf
-        m_use = m_new;
-      }
-      // p = 2^(cl*s - mc), two lanes per instruction; pairs (c2 & 7) < kEmuPer8 go to the
-      // FMA-pipe polynomial, the rest to the MUFU ex2
-      const float mc = m_use * cl - C::kPShift;
-      const uint64_t cl2 = f2_pack(cl, cl), nmc2 = f2_pack(-mc, -mc);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-      // Two halves of 32 column pairs; each half's P words go to TMEM as soon as they are
-      // complete, so their registers (and the scores they came from) are free for the rest.
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pw[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int c2 = half * 32 + i;
-          const uint64_t x =
-              f2_fma(f2_pack(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), cl2, nmc2);
-          float x0, x1, e0, e1;
-          f2_unpack(x, x0, x1);
-          if ((c2 & 7) < C::kEmuPer8) {
-            exp2_fma2(x0, x1, e0, e1);
-          } else {
-            e0 = ex2_approx(x0);
-            e1 = ex2_approx(x1);
-          }
-          acc[c2 & 3] = f2_add(acc[c2 & 3], f2_pack(e0, e1));
-          if constexpr (!FP8) {
-            pw[i] = pack_bf16x2(e0, e1);
-          } else {
-            // four e4m3 per TMEM column: pair 2q in bytes 0-1, pair 2q+1 in bytes 2-3
-            const uint32_t h = pack_e4m3x2(e0, e1);
-            if (i & 1) pw[i >> 1] |= h << 16;
-            else pw[i >> 1] = h;
-          }
-        }
-        if constexpr (!FP8) {
-          tmem_st32(tS + 32 * half, pw);
-        } else {
-          tmem_st16(tS + 16 * half, *reinterpret_cast<uint32_t(*)[16]>(pw));
-        }
-      }
+      if (valid < C::kBN) mask_tail(s, valid);
+      // Speculative pass (bf16): exponentiate with the running max m_use and keep the result
+      // when the row sum shows that no p exceeds the lazy-rescale bound (every p <= sum <=
+      // kSumBound), the usual case after the first tile.  Otherwise (first tile, a row max
+      // that rose a lot, or the e4m3 path) the warp takes the exact route: (re)load S (still
+      // intact in TMEM, P is not written yet), exact row max, rescale, exponentiate.
+      uint32_t pw[2 * C::kPWordsHalf];
       float sum;
-      {
-        const uint64_t a01 = f2_add(acc[0], acc[1]), a23 = f2_add(acc[2], acc[3]);
-        float lo, hi;
-        f2_unpack(f2_add(a01, a23), lo, hi);
-        sum = lo + hi;
+      float alpha = 1.0f;
+      bool need = false;
+      bool slow = (j == 0) || !C::kSpeculative;
+      if (!slow) {
+        exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
+        slow = __any_sync(0xffffffffu, !(sum <= C::kSumBound));
       }
+      if (slow) {
+        if (j > 0 && C::kSpeculative) {
+          tmem_ld128_sync(tS, s);
+          if (valid < C::kBN) mask_tail(s, valid);
+        }
+        const float m_new = fmaxf(m_use, row_max128(s));
+        need = (m_new - m_use) * cl > C::kRescaleLog2;       // true on the first tile
+        if (need) {
+          alpha = ex2_approx((m_use - m_new) * cl);          // 0 when m_use = -inf
+          m_use = m_new;
+        }
+        exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
+      }
+      tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
+      if constexpr (!FP8) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
       tmem_st_wait();
       // O_t is quiescent here (PV_t(j-1) completed before S_t(j) was signalled).
       if (j > 0 && __any_sync(0xffffffffu, need)) {
