@@ -316,6 +316,7 @@ def run_ours(args, rank, local_rank, world):
     # end to end through the C ABI with host buffers: pinned H2D of Q, K, V, the step, D2H of
     # the outputs, all inside the timed region
     e2e = run_e2e(args, lsa, step, data, stream, dev, ranks)
+    ring = run_ring_fused(lsa, step, stream, ranks) if step.bounds else None
 
     ranks.close()
     if rank != 0:
@@ -369,11 +370,45 @@ def run_ours(args, rank, local_rank, world):
                                   "algorithmic_bytes": mbytes}
     if fp8_ms:
         line["fp8_fwd_tflops"] = round(w.flops / (statistics.mean(fp8_ms) * 1e-3) / 1e12, 2)
+    if ring is not None:
+        ring["chunks_plus_merge_ms"] = round((statistics.mean(chunk_ms) + statistics.mean(merge_ms)), 4)
+        line["ring_fused"] = ring
     line["clocks"] = clk.summary()
     line["e2e"] = e2e
     if world == 1 and not args.skip_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def run_ring_fused(lsa, step, stream, ranks, reps: int = 10):
+    """The same chunked pass with fused ring steps: dit_attn_acc_init + n x
+    dit_attn_fwd_chunk_acc into an fp32 accumulator (reported beside the step, not in it)."""
+    import torch
+    w = step.w
+    B, H, S, D = w.B, w.H, w.S, w.D
+    acc = torch.empty((B, H, S, D), dtype=torch.float32, device=step.q.device)
+    acc_lse = torch.empty((B, H, S), dtype=torch.float32, device=step.q.device)
+
+    def one():
+        lsa.dit_attn_acc_init(acc, acc_lse, B, H, S, D, stream)
+        for a, b in step.bounds:
+            lsa.dit_attn_fwd_chunk_acc(step.q, step.k, step.v, acc, acc_lse, B, H, S, S, D, a, b, w.scale,
+                                       lsa.DIT_BF16, None, stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            one()
+        stream.synchronize()
+        ranks.barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            one()
+        t1.record(stream)
+    stream.synchronize()
+    ms = ranks.max(t0.elapsed_time(t1)) / reps
+    return {"ms": round(ms, 4), "tflops": round(w.flops * ranks.world / (ms * 1e-3) / 1e12, 2),
+            "calls": "dit_attn_acc_init + %d x dit_attn_fwd_chunk_acc" % len(step.bounds)}
 
 
 def run_e2e(args, lsa, step, data, stream, dev, ranks):

@@ -88,6 +88,32 @@ int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, f
                        int out_dtype, const float* descale_qkv, void* stream);
 
 /*
+ * dit_attn_fwd_chunk_acc - one ring step fused into the forward: attention of the S_q queries
+ * against the keys k0 <= j < k1, merged in the epilogue into a running accumulator
+ *     lse' = log(exp(acc_lse) + exp(lse_c)),
+ *     acc_out' = (exp(acc_lse - lse') acc_out + exp(lse_c - lse') out_c)
+ * (the same exact combination as dit_attn_merge, applied pairwise), so a ring of chunks needs
+ * no stored partials and no separate merge launch.  This is the per-block step of the USP
+ * Ring dimension (xDiT overview page, section 3.2.2), on one GPU.
+ *
+ *   acc_out   [B,H,S_q,D] fp32, read and written (16-byte aligned).
+ *   acc_lse   [B,H,S_q] fp32, read and written.  An accumulator with acc_lse = -inf (and any
+ *             acc_out) is empty: see dit_attn_acc_init.  The first chunk may also be written
+ *             by dit_attn_fwd_chunk with out_dtype = DIT_FP32.
+ *   Other arguments as for dit_attn_fwd_chunk.  k0 == k1 leaves the accumulator unchanged.
+ *   Calls that update the same accumulator must be ordered (same stream, or events).
+ *   The final bf16 output can be produced with dit_attn_merge(n_chunks = 1).
+ */
+int dit_attn_fwd_chunk_acc(const void* q, const void* k, const void* v, float* acc_out, float* acc_lse,
+                           int B, int H, int S_q, int S_kv, int D, int k0, int k1, float scale,
+                           int dtype, const float* descale_qkv, void* stream);
+
+/*
+ * dit_attn_acc_init - empty accumulator: acc_out = 0, acc_lse = -inf ([B,H,S,D] / [B,H,S] fp32).
+ */
+int dit_attn_acc_init(float* acc_out, float* acc_lse, int B, int H, int S, int D, void* stream);
+
+/*
  * dit_attn_merge - exact log-sum-exp combination of n_chunks partials (out_c, lse_c):
  *     M = max_c lse_c, w_c = exp(lse_c - M), L = sum_c w_c,
  *     lse = M + log L, out = sum_c (w_c / L) out_c;  all lse_c = -inf -> out = 0, lse = -inf.

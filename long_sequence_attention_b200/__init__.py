@@ -42,6 +42,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, f, i, vp, vp]
     lib.dit_attn_fwd_chunk.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, i, vp, vp]
     lib.dit_attn_merge.argtypes = [ctypes.POINTER(vp), ctypes.POINTER(vp), i, vp, vp, i, i, i, i, i, i, vp]
+    lib.dit_attn_fwd_chunk_acc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp, vp]
+    lib.dit_attn_acc_init.argtypes = [vp, vp, i, i, i, i, vp]
     lib.dit_quant_fp8_workspace_bytes.argtypes = [ll]
     lib.dit_quant_fp8_workspace_bytes.restype = sz
     lib.dit_quant_fp8.argtypes = [vp, vp, vp, ll, vp, sz, vp]
@@ -53,7 +55,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
     lib.dit_version.argtypes = []
-    for name in ("dit_attn_fwd", "dit_attn_fwd_chunk", "dit_attn_merge", "dit_quant_fp8", "dit_device_status",
+    for name in ("dit_attn_fwd", "dit_attn_fwd_chunk", "dit_attn_fwd_chunk_acc", "dit_attn_acc_init",
+                 "dit_attn_merge", "dit_quant_fp8", "dit_device_status",
                  "dit_set_wait_timeout_us", "dit_selftest_wait_timeout", "dit_version"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
@@ -102,6 +105,17 @@ def dit_attn_fwd_chunk(q, k, v, out, lse, B: int, H: int, S_q: int, S_kv: int, D
     _check(lib.dit_attn_fwd_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S_q, S_kv, D, k0, k1,
                                   float(scale), dtype, out_dtype, _ptr(descale_qkv), _stream(stream)),
            "dit_attn_fwd_chunk")
+
+
+def dit_attn_fwd_chunk_acc(q, k, v, acc_out, acc_lse, B: int, H: int, S_q: int, S_kv: int, D: int, k0: int,
+                           k1: int, scale: float, dtype: int = DIT_BF16, descale_qkv=None, stream=None) -> None:
+    _check(lib.dit_attn_fwd_chunk_acc(_ptr(q), _ptr(k), _ptr(v), _ptr(acc_out), _ptr(acc_lse), B, H, S_q, S_kv, D,
+                                      k0, k1, float(scale), dtype, _ptr(descale_qkv), _stream(stream)),
+           "dit_attn_fwd_chunk_acc")
+
+
+def dit_attn_acc_init(acc_out, acc_lse, B: int, H: int, S: int, D: int, stream=None) -> None:
+    _check(lib.dit_attn_acc_init(_ptr(acc_out), _ptr(acc_lse), B, H, S, D, _stream(stream)), "dit_attn_acc_init")
 
 
 def dit_attn_merge(outs: Sequence, lses: Sequence, out, lse, B: int, H: int, S: int, D: int,
@@ -182,6 +196,23 @@ def attention_chunk(q, k, v, k0: int, k1: int, scale: Optional[float] = None, ou
     dit_attn_fwd_chunk(q, k, v, out, lse, B, H, S_q, S_kv, D, k0, k1, scale,
                        DIT_FP8_E4M3 if fp8 else DIT_BF16, DIT_FP32 if od == torch.float32 else DIT_BF16,
                        descale_qkv, stream)
+    return out, lse
+
+
+def ring_attention(q, k, v, bounds: Sequence, scale: Optional[float] = None, descale_qkv=None, stream=None):
+    """Attention accumulated over the KV ranges in `bounds` with fused ring steps:
+    (out fp32, lse) = exact attention over the union of the ranges."""
+    import torch
+    B, H, S_q, D = _dims(q)
+    S_kv = int(k.shape[2])
+    fp8 = q.dtype == torch.uint8
+    scale = (1.0 / D ** 0.5) if scale is None else scale
+    out = torch.empty((B, H, S_q, D), dtype=torch.float32, device=q.device)
+    lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q.device)
+    dit_attn_acc_init(out, lse, B, H, S_q, D, stream)
+    for k0, k1 in bounds:
+        dit_attn_fwd_chunk_acc(q, k, v, out, lse, B, H, S_q, S_kv, D, k0, k1, scale,
+                               DIT_FP8_E4M3 if fp8 else DIT_BF16, descale_qkv, stream)
     return out, lse
 
 

@@ -61,6 +61,7 @@ struct AttnParams {
   void* out;               // [B,H,S_q,D] bf16 or fp32
   float* lse;              // [B,H,S_q] natural-log LSE, may be null
   int out_fp32;
+  int accumulate;          // 1: out (fp32) and lse hold a running (O, LSE); merge this range into them
   unsigned long long timeout_ns;
 };
 
@@ -497,14 +498,41 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const int grow = q_start + t * C::kBM + row;
       const bool store = grow < p.S_q;
-      const float inv_l = dv / l;
-      const size_t row_elem = (static_cast<size_t>(bh) * p.S_q + grow) * D;
+      const size_t row_idx = static_cast<size_t>(bh) * p.S_q + grow;
+      const size_t row_elem = row_idx * D;
+      const float lse_c = scale_eff * m_use + logf(l) - C::kPShift * 0.6931471805599453f;
+      // Accumulate mode (one ring step): (O, LSE) <- exact LSE merge of the running pair and
+      // this range's partial, w = exp(lse - M) / L with M the larger LSE and L the weight sum.
+      float w_old = 0.0f, w_new = 1.0f, lse_out = lse_c;
+      if (p.accumulate && store) {
+        const float la = p.lse[row_idx];
+        const float M = fmaxf(la, lse_c);
+        const float ea = __expf(la - M);                     // 0 for an empty accumulator
+        const float ec = __expf(lse_c - M);
+        const float L = ea + ec;
+        w_old = ea / L;
+        w_new = ec / L;
+        lse_out = M + logf(L);
+      }
+      const float inv_l = dv / l * w_new;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
         tmem_ld32_sync(tO + cc * 32, o);
         if (store) {
-          if (p.out_fp32) {
+          if (p.accumulate && w_old != 0.0f) {
+            // (an empty accumulator, w_old = 0, is overwritten below without being read, so
+            // whatever its buffer holds cannot leak in)
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_elem + cc * 32);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 a = dst[i];
+              dst[i] = make_float4(fmaf(a.x, w_old, __uint_as_float(o[4 * i]) * inv_l),
+                                   fmaf(a.y, w_old, __uint_as_float(o[4 * i + 1]) * inv_l),
+                                   fmaf(a.z, w_old, __uint_as_float(o[4 * i + 2]) * inv_l),
+                                   fmaf(a.w, w_old, __uint_as_float(o[4 * i + 3]) * inv_l));
+            }
+          } else if (p.out_fp32 || p.accumulate) {
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_elem + cc * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -521,9 +549,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
       }
-      if (store && p.lse != nullptr)
-        p.lse[static_cast<size_t>(bh) * p.S_q + grow] =
-            scale_eff * m_use + logf(l) - C::kPShift * 0.6931471805599453f;
+      if (store && p.lse != nullptr) p.lse[row_idx] = lse_out;
       // The O reads above end with tcgen05.wait::ld; the next unit's first P.V (which
       // overwrites O_t) is issued only after this warpgroup publishes that unit's P_t.
     }

@@ -191,11 +191,11 @@ int noalloc_scratch(float** out) {
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
-                       int S_q, int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
-                       const float* descale_qkv, void* stream) {
+int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S_q,
+                    int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
+                    const float* descale_qkv, void* stream, bool accumulate) {
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || S_q < 1 || S_kv < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (k0 < 0 || k1 < k0 || k1 > S_kv) return DIT_ERR_INVALID_ARG;
@@ -222,6 +222,7 @@ int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, f
     return DIT_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
+  if (accumulate && k0 == k1) return DIT_OK;   // merging an empty range changes nothing
   if (k0 == k1) {
     const long long rows = static_cast<long long>(rows_q);
     attn_fill_empty_kernel<<<grid_for(rows * D, 256, 148 * 16), 256, 0, st>>>(out, lse, rows, D,
@@ -236,10 +237,42 @@ int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, f
   prm.out = out;
   prm.lse = lse;
   prm.out_fp32 = out_dtype == DIT_FP32;
+  prm.accumulate = accumulate ? 1 : 0;
   prm.timeout_ns = g_timeout_ns.load();
   if (fp8) return launch_attn<128, true>(q, k, v, prm, st);
   if (D == 64) return launch_attn<64, false>(q, k, v, prm, st);
   return launch_attn<128, false>(q, k, v, prm, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int dit_attn_fwd_chunk(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                       int S_q, int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
+                       const float* descale_qkv, void* stream) {
+  return attn_chunk_impl(q, k, v, out, lse, B, H, S_q, S_kv, D, k0, k1, scale, dtype, out_dtype, descale_qkv,
+                         stream, false);
+}
+
+int dit_attn_fwd_chunk_acc(const void* q, const void* k, const void* v, float* acc_out, float* acc_lse, int B,
+                           int H, int S_q, int S_kv, int D, int k0, int k1, float scale, int dtype,
+                           const float* descale_qkv, void* stream) {
+  if (acc_out == nullptr || acc_lse == nullptr) return DIT_ERR_INVALID_ARG;
+  return attn_chunk_impl(q, k, v, acc_out, acc_lse, B, H, S_q, S_kv, D, k0, k1, scale, dtype, DIT_FP32,
+                         descale_qkv, stream, true);
+}
+
+int dit_attn_acc_init(float* acc_out, float* acc_lse, int B, int H, int S, int D, void* stream) {
+  if (acc_out == nullptr || acc_lse == nullptr || B < 1 || H < 1 || S < 1) return DIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned(acc_out, 16) || !aligned(acc_lse, 4)) return DIT_ERR_MISALIGNED;
+  const long long rows = static_cast<long long>(B) * H * S;
+  if (overlaps(acc_out, static_cast<size_t>(rows) * D * 4, acc_lse, static_cast<size_t>(rows) * 4))
+    return DIT_ERR_INVALID_ARG;
+  attn_fill_empty_kernel<<<grid_for(rows * D, 256, 148 * 16), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      acc_out, acc_lse, rows, D, 1);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
 int dit_attn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S,
