@@ -185,6 +185,16 @@ int dit_device_status(int* status, int clear);
 int dit_set_wait_timeout_us(unsigned long long timeout_us);
 
 /*
+ * dit_set_sm_reserve - process-wide number of SMs that the attention kernels leave free
+ * (default 0).  The attention forward is a persistent kernel with one CTA per SM that fills
+ * each SM's shared memory and registers, so no other kernel can run beside it; a KV ring
+ * whose NCCL send/recv kernels should overlap the attention of the current block reserves
+ * a few SMs for them.  The grid is max(1, SMs - n_sms) CTAs at most; results do not depend
+ * on it.  0 <= n_sms <= 1024, else DIT_ERR_INVALID_ARG.
+ */
+int dit_set_sm_reserve(int n_sms);
+
+/*
  * dit_selftest_wait_timeout - enqueues a one-thread kernel that waits on a barrier nothing
  * ever arrives at, with the given limit, so the caller can check that the bounded wait
  * gives up and that dit_device_status() then reports DIT_ERR_TIMEOUT.

@@ -52,6 +52,7 @@ def _load() -> ctypes.CDLL:
     lib.dit_device_status.argtypes = [ctypes.POINTER(i), i]
     lib.dit_set_wait_timeout_us.argtypes = [ull]
     lib.dit_selftest_wait_timeout.argtypes = [ull, vp]
+    lib.dit_set_sm_reserve.argtypes = [i]
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
     lib.dit_version.argtypes = []
@@ -151,6 +152,10 @@ def dit_device_status(clear: bool = True) -> int:
 
 def dit_set_wait_timeout_us(us: int) -> None:
     _check(lib.dit_set_wait_timeout_us(int(us)), "dit_set_wait_timeout_us")
+
+
+def dit_set_sm_reserve(n_sms: int) -> None:
+    _check(lib.dit_set_sm_reserve(int(n_sms)), "dit_set_sm_reserve")
 
 
 def dit_selftest_wait_timeout(timeout_us: int, stream=None) -> None:

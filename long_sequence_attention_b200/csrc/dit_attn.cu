@@ -19,6 +19,7 @@ namespace {
 using namespace dit;
 
 std::atomic<unsigned long long> g_timeout_ns{1000000000ull};
+std::atomic<int> g_sm_reserve{0};   // SMs the persistent attention grid leaves free
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -131,7 +132,10 @@ int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p
   pr.n_units = pr.n_qblk * prm.H * prm.B;
   int sms = 0;
   if ((rc = sm_count(&sms)) != DIT_OK) return rc;
-  const int grid = pr.n_units < sms ? pr.n_units : sms;   // persistent: at most one CTA per SM
+  // persistent: at most one CTA per SM, minus the SMs reserved for concurrent kernels
+  const int reserve = g_sm_reserve.load();
+  const int slots = sms - reserve > 1 ? sms - reserve : 1;
+  const int grid = pr.n_units < slots ? pr.n_units : slots;
   attn_fwd_kernel<D, FP8><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, pr);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
@@ -377,6 +381,12 @@ int dit_device_status(int* status, int clear) {
 
 int dit_set_wait_timeout_us(unsigned long long timeout_us) {
   g_timeout_ns.store(timeout_us == 0 ? 1000000000ull : timeout_us * 1000ull);
+  return DIT_OK;
+}
+
+int dit_set_sm_reserve(int n_sms) {
+  if (n_sms < 0 || n_sms > 1024) return DIT_ERR_INVALID_ARG;
+  g_sm_reserve.store(n_sms);
   return DIT_OK;
 }
 

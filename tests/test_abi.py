@@ -126,3 +126,10 @@ def test_quant_validation(lib):
 def test_selftest_validation(lib):
     assert lib.lib.dit_selftest_wait_timeout(0, None) == 1
     assert lib.lib.dit_selftest_wait_timeout(10 ** 9, None) == 1
+
+
+def test_sm_reserve_validation(lib):
+    assert lib.lib.dit_set_sm_reserve(-1) == 1
+    assert lib.lib.dit_set_sm_reserve(1025) == 1
+    assert lib.lib.dit_set_sm_reserve(8) == 0
+    assert lib.lib.dit_set_sm_reserve(0) == 0

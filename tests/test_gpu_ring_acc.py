@@ -107,3 +107,47 @@ def test_acc_argument_validation(cuda_lib):
     assert f(x.data_ptr(), x.data_ptr(), x.data_ptr(), a.data_ptr(), l.data_ptr(), 1, 1, 64, 64, 64, 10, 5, 0.1, 0,
              None, None) == 1
     assert cuda_lib.lib.dit_attn_acc_init(a.data_ptr(), l.data_ptr(), 1, 1, 64, 96, None) == 2
+
+
+def test_sm_reserve_leaves_results_bit_identical(cuda_lib):
+    """A smaller persistent grid (SMs reserved for concurrent kernels) processes the same work
+    units in another order per CTA; every unit's arithmetic is unchanged."""
+    import torch
+    host, dev = _case(2, 3, 900, 900, 128, seed=5)
+    ref_o, ref_l = cuda_lib.attention(*dev, 0.09)
+    try:
+        cuda_lib.dit_set_sm_reserve(140)
+        o, l = cuda_lib.attention(*dev, 0.09)
+        torch.cuda.synchronize()
+    finally:
+        cuda_lib.dit_set_sm_reserve(0)
+    assert torch.equal(o, ref_o) and torch.equal(l, ref_l)
+    with pytest.raises(cuda_lib.DitError):
+        cuda_lib.dit_set_sm_reserve(-1)
+
+
+@pytest.mark.parametrize("out_bf16", [False, True])
+def test_ring_driver_single_rank_nccl(cuda_lib, out_bf16):
+    """The multi-rank ring driver on a one-rank NCCL group: one fused step over the local
+    block (the send/recv schedule itself is covered by the gloo tests on CPU)."""
+    import datetime
+    import socket
+    import torch
+    import torch.distributed as dist
+    from long_sequence_attention_b200.ring import ring_attention_dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=30))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        host, dev = _case(1, 4, 333, 333, 128, seed=8)
+        out, lse = ring_attention_dist(*dev, 0.1, out_dtype=torch.bfloat16 if out_bf16 else None)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert out.dtype == (torch.bfloat16 if out_bf16 else torch.float32)
+    ro, rl = oracle.attention(*host, 0.1)
+    m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
+    assert_bf16_parity(m, out_bf16)
