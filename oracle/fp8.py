@@ -17,6 +17,10 @@ the FP8 layout or the scaling; the readings used here:
 * Per-tensor scale: amax = max |x|; descale = amax / 448 in float32 (descale = 1
   when amax = 0); codes = encode(float32(x) / descale) with an IEEE float32 division.
   The dequantised value is decode(code) * descale.
+* Per-block scale (a finer variant of the same scheme, not described by the pages): a
+  [B,H,S,D] tensor is cut, per (b, h), into blocks of 128 consecutive rows (tokens), the
+  last one ragged; each block is quantised exactly as a tensor of its own, with its own
+  descale.  Descales form a float32 [B,H,ceil(S/128)] array.
 """
 
 from __future__ import annotations
@@ -86,3 +90,29 @@ def quantize_per_tensor(x: np.ndarray) -> Tuple[np.ndarray, np.float32]:
 def dequantize(codes: np.ndarray, descale: float) -> np.ndarray:
     """decode(code) * descale in float64."""
     return e4m3_decode(codes) * float(np.float32(descale))
+
+
+BLOCK_ROWS = 128
+
+
+def quantize_per_block(x: np.ndarray, block_rows: int = BLOCK_ROWS) -> Tuple[np.ndarray, np.ndarray]:
+    """(codes uint8 [B,H,S,D], descales float32 [B,H,nblk]) for a [B,H,S,D] tensor: every
+    run of block_rows rows of one (b, h) is quantised per tensor on its own."""
+    x32 = np.asarray(x, dtype=np.float32)
+    B, H, S, D = x32.shape
+    nblk = (S + block_rows - 1) // block_rows
+    codes = np.empty(x32.shape, dtype=np.uint8)
+    descales = np.empty((B, H, nblk), dtype=np.float32)
+    for b in range(B):
+        for h in range(H):
+            for i in range(nblk):
+                rows = slice(i * block_rows, min(S, (i + 1) * block_rows))
+                codes[b, h, rows], descales[b, h, i] = quantize_per_tensor(x32[b, h, rows])
+    return codes, descales
+
+
+def dequantize_per_block(codes: np.ndarray, descales: np.ndarray, block_rows: int = BLOCK_ROWS) -> np.ndarray:
+    """decode(code) * descale of the code's block, in float64."""
+    S = codes.shape[2]
+    per_row = np.repeat(np.asarray(descales, dtype=np.float32).astype(np.float64), block_rows, axis=2)[:, :, :S]
+    return e4m3_decode(codes) * per_row[..., None]

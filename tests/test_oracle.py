@@ -391,3 +391,51 @@ def test_quantize_per_tensor():
     assert np.max(np.abs(deq)) == pytest.approx(amax, rel=2 ** -4)
     zc, zd = fp8.quantize_per_tensor(np.zeros(10, dtype=np.float32))
     assert zd == 1.0 and np.all(zc == 0)
+
+
+def test_quantize_per_block_constructed_scales():
+    """Block i of each (b, h) holds E4M3-exact values times 2^i with 448 * 2^i present, so its
+    descale is exactly 2^i and its codes are the plain encodings of the pattern; the ragged
+    last block (S = 2 * 128 + 5) and an all-zero block follow the same rule."""
+    rng = np.random.default_rng(3)
+    B, H, S, D = 2, 3, 2 * 128 + 5, 16
+    pos = fp8.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    pattern_codes = rng.integers(0, 0x7F, size=(B, H, S, D)).astype(np.uint8)
+    pattern_codes |= (rng.integers(0, 2, size=pattern_codes.shape) << 7).astype(np.uint8)
+    pattern_codes[:, :, ::128, 0] = 0x7E                  # 448 in every block
+    x = fp8.e4m3_decode(pattern_codes)
+    for i in range(3):
+        x[:, :, i * 128:(i + 1) * 128] *= 2.0 ** i
+    x[1, 2, 128:256] = 0.0                                 # one all-zero block
+    codes, ds = fp8.quantize_per_block(x.astype(np.float32))
+    want_ds = np.broadcast_to(np.array([1.0, 2.0, 4.0], dtype=np.float32), (B, H, 3)).copy()
+    want_ds[1, 2, 1] = 1.0
+    assert ds.dtype == np.float32 and np.array_equal(ds, want_ds)
+    want_codes = pattern_codes.copy()
+    want_codes[1, 2, 128:256] = np.where(np.signbit(x[1, 2, 128:256]), 0x80, 0x00)
+    assert np.array_equal(codes, want_codes)
+    assert np.array_equal(fp8.dequantize_per_block(codes, ds), x)
+    assert np.all(np.isin(pos, pos))
+
+
+def test_quantize_per_block_is_per_tensor_on_each_block():
+    """Each block's codes and descale equal a per-tensor quantisation of that block alone, and
+    one block covering all rows is the per-tensor quantiser itself."""
+    x = make_tensor((1, 2, 300, 8), 11) * np.float32(5.0)
+    x[0, 1, 150:170] *= np.float32(1e5)                     # an outlier run in block 1 of head 1
+    codes, ds = fp8.quantize_per_block(x)
+    assert ds.shape == (1, 2, 3)
+    for h in range(2):
+        for i, (a, b) in enumerate([(0, 128), (128, 256), (256, 300)]):
+            c1, d1 = fp8.quantize_per_tensor(x[0, h, a:b])
+            assert d1 == ds[0, h, i] and np.array_equal(c1, codes[0, h, a:b])
+    cw, dw = fp8.quantize_per_block(x[:, :1], block_rows=300)
+    ct, dt = fp8.quantize_per_tensor(x[:, :1])
+    assert dw[0, 0, 0] == dt and np.array_equal(cw, ct)
+    # the outlier run pushes head 0 into the subnormal codes under one per-tensor scale; with
+    # block scales head 0 keeps E4M3's relative step (rel-L2 about 2^-5)
+    ct2, dt2 = fp8.quantize_per_tensor(x)
+
+    def rel(a):
+        return np.linalg.norm(a[0, 0] - x[0, 0]) / np.linalg.norm(x[0, 0])
+    assert rel(fp8.dequantize_per_block(codes, ds)) < 0.05 and rel(fp8.dequantize(ct2, dt2)) > 0.2
