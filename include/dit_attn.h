@@ -145,6 +145,36 @@ int dit_quant_fp8(const void* x_bf16, void* x_fp8, float* descale, long long n, 
                   size_t workspace_bytes, void* stream);
 
 /*
+ * dit_quant_fp8_blocks - per-block E4M3 quantisation: every run of 128 consecutive rows
+ * (tokens) of one (b, h) of a [B,H,S,D] bf16 tensor is quantised as a tensor of its own
+ * (the rule of dit_quant_fp8), the last run of a head ragged when S % 128 != 0.  A finer
+ * variant of the per-tensor scheme for inputs whose magnitude varies along the sequence; the
+ * pages fix no FP8 scaling scheme.  An all-zero block records descale 0 and zero codes.
+ *
+ *   x_bf16    [B,H,S,D] bf16 (16-byte aligned);  x_fp8  [B,H,S,D] E4M3 codes (8-byte aligned).
+ *   descales  [B,H,ceil(S/128)] fp32, written.  8 <= D <= 128, D % 8 == 0.
+ *   One kernel launch; each element is read and written once.
+ */
+int dit_quant_fp8_blocks(const void* x_bf16, void* x_fp8, float* descales, int B, int H, int S, int D,
+                         void* stream);
+
+/*
+ * dit_attn_fwd_fp8_blocks - dit_attn_fwd_chunk on E4M3 inputs quantised per block by
+ * dit_quant_fp8_blocks: q_ij = code * dq_blk[b,h,i/128], likewise k and v.
+ *
+ *   q8, k8, v8  [B,H,S_q,D] / [B,H,S_kv,D] E4M3 codes.
+ *   dq_blk      [B,H,ceil(S_q/128)] fp32;  dk_blk, dv_blk  [B,H,ceil(S_kv/128)] fp32.
+ *   D = 128.  k0 must be a multiple of 128 (each 128-key tile has one scale), else
+ *   DIT_ERR_UNSUPPORTED.  Other arguments and results as for dit_attn_fwd_chunk.
+ *   In the kernel, Q and K scales enter the softmax scale of each tile pair; V scales enter
+ *   P as ratios descale_v(j) / max_j descale_v(j) <= 1 and the maximum is applied to O.
+ */
+int dit_attn_fwd_fp8_blocks(const void* q8, const void* k8, const void* v8, const float* dq_blk,
+                            const float* dk_blk, const float* dv_blk, void* out, float* lse, int B,
+                            int H, int S_q, int S_kv, int D, int k0, int k1, float scale,
+                            int out_dtype, void* stream);
+
+/*
  * dit_quant_fp8_noalloc - the same quantisation as dit_quant_fp8, for callers that cannot
  * allocate device memory: code that runs where cudaMalloc is off limits (for example while
  * a stream is being captured into a CUDA graph, or inside a framework whose allocator owns

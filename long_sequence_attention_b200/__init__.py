@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_set_wait_timeout_us.argtypes = [ull]
     lib.dit_selftest_wait_timeout.argtypes = [ull, vp]
     lib.dit_set_sm_reserve.argtypes = [i]
+    lib.dit_quant_fp8_blocks.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    lib.dit_attn_fwd_fp8_blocks.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
     lib.dit_version.argtypes = []
@@ -135,6 +137,18 @@ def dit_quant_fp8_workspace_bytes(n: int) -> int:
 def dit_quant_fp8(x_bf16, x_fp8, descale, n: int, workspace, workspace_bytes: int, stream=None) -> None:
     _check(lib.dit_quant_fp8(_ptr(x_bf16), _ptr(x_fp8), _ptr(descale), int(n), _ptr(workspace),
                              int(workspace_bytes), _stream(stream)), "dit_quant_fp8")
+
+
+def dit_quant_fp8_blocks(x_bf16, x_fp8, descales, B: int, H: int, S: int, D: int, stream=None) -> None:
+    _check(lib.dit_quant_fp8_blocks(_ptr(x_bf16), _ptr(x_fp8), _ptr(descales), B, H, S, D, _stream(stream)),
+           "dit_quant_fp8_blocks")
+
+
+def dit_attn_fwd_fp8_blocks(q8, k8, v8, dq_blk, dk_blk, dv_blk, out, lse, B: int, H: int, S_q: int, S_kv: int,
+                            D: int, k0: int, k1: int, scale: float, out_dtype: int = 0, stream=None) -> None:
+    _check(lib.dit_attn_fwd_fp8_blocks(_ptr(q8), _ptr(k8), _ptr(v8), _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk),
+                                       _ptr(out), _ptr(lse), B, H, S_q, S_kv, D, k0, k1, float(scale), out_dtype,
+                                       _stream(stream)), "dit_attn_fwd_fp8_blocks")
 
 
 def dit_quant_fp8_noalloc(x_bf16, x_fp8, descale, n: int, stream=None) -> None:
@@ -230,6 +244,32 @@ def merge(outs: Sequence, lses: Sequence, out_dtype=None, stream=None):
     lse = torch.empty((B, H, S), dtype=torch.float32, device=outs[0].device)
     in_dt = DIT_FP32 if outs[0].dtype == torch.float32 else DIT_BF16
     dit_attn_merge(outs, lses, out, lse, B, H, S, D, in_dt, DIT_FP32 if od == torch.float32 else DIT_BF16, stream)
+    return out, lse
+
+
+def quantize_fp8_blocks(x, stream=None):
+    """(codes uint8 [B,H,S,D], descales fp32 [B,H,ceil(S/128)]) of a bf16 [B,H,S,D] tensor."""
+    import torch
+    B, H, S, D = _dims(x)
+    codes = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    ds = torch.empty((B, H, (S + 127) // 128), dtype=torch.float32, device=x.device)
+    dit_quant_fp8_blocks(x, codes, ds, B, H, S, D, stream)
+    return codes, ds
+
+
+def attention_fp8_blocks(q8, k8, v8, dq, dk, dv, scale: Optional[float] = None, k0: int = 0, k1: Optional[int] = None,
+                         out_dtype=None, stream=None):
+    """(out, lse) of E4M3 inputs with per-block descales over keys [k0, k1)."""
+    import torch
+    B, H, S_q, D = _dims(q8)
+    S_kv = int(k8.shape[2])
+    k1 = S_kv if k1 is None else k1
+    scale = (1.0 / D ** 0.5) if scale is None else scale
+    odt = torch.bfloat16 if out_dtype is None else out_dtype
+    out = torch.empty((B, H, S_q, D), dtype=odt, device=q8.device)
+    lse = torch.empty((B, H, S_q), dtype=torch.float32, device=q8.device)
+    dit_attn_fwd_fp8_blocks(q8, k8, v8, dq, dk, dv, out, lse, B, H, S_q, S_kv, D, k0, k1, scale,
+                            DIT_FP32 if odt == torch.float32 else DIT_BF16, stream)
     return out, lse
 
 

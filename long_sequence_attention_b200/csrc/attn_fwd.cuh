@@ -62,6 +62,12 @@ struct AttnParams {
   float* lse;              // [B,H,S_q] natural-log LSE, may be null
   int out_fp32;
   int accumulate;          // 1: out (fp32) and lse hold a running (O, LSE); merge this range into them
+  // e4m3 with per-block scales (else null): descales of 128-row blocks per (b, h),
+  // dq_blk [B*H, nb_q], dk_blk / dv_blk [B*H, nb_kv]; k0 is then a multiple of 128
+  const float* dq_blk;
+  const float* dk_blk;
+  const float* dv_blk;
+  int nb_q, nb_kv;
   unsigned long long timeout_ns;
 };
 
@@ -425,18 +431,61 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem_base + lane_off + (t ? C::kColS1 : C::kColS0);
     const uint32_t tO = tmem_base + lane_off + (t ? C::kColO1 : C::kColO0);
 
+    // Scales.  bf16: scores in raw units, cl = scale * log2(e) turns them into log2 units.
+    // e4m3: the running max is kept in log2 units, and every KV tile j has its own
+    //   cl_j = scale * descale_q(tile) * descale_k(j) * log2(e)
+    // (one value for all tiles with per-tensor scales).  With per-block V scales, tile j's
+    // P is stored as p * r_j, r_j = descale_v(j) / dv_out (dv_out = the largest V descale of
+    // the range, so r_j <= 1 and P stays in range), which puts descale_v(j) / dv_out into
+    // the P.V products; the epilogue multiplies by dv_out.  The row sum uses p itself: the
+    // sum of the stored values divided by r_j.
     float dq = 1.0f, dk = 1.0f, dv = 1.0f;
-    if constexpr (FP8) { dq = p.descale[0]; dk = p.descale[1]; dv = p.descale[2]; }
+    const bool blk = FP8 && p.dk_blk != nullptr;
+    if constexpr (FP8) {
+      if (!blk) { dq = p.descale[0]; dk = p.descale[1]; dv = p.descale[2]; }
+    }
     const float scale_eff = p.scale * dq * dk;                 // natural-log units per raw score
     const float cl = scale_eff * 1.4426950408889634f;          // log2 units per raw score
     bool ok = true;
 
     for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
     const int bh = unit_bh(u), q_start = unit_q0(u);
-    float m_use = -INFINITY;                                   // running (lazy) max, raw units
+    float m_use = -INFINITY;             // running (lazy) max: raw units (bf16), log2 units (e4m3)
     float l = 0.0f;
+    float cl_q = cl, dv_out = dv;        // per unit and Q tile (e4m3 per-block scales)
+    float dk_nxt = dk, dv_nxt = dv;      // descales of the next KV tile, loaded one tile ahead
+    if constexpr (FP8) {
+      if (blk) {
+        const int bq = min((q_start + t * C::kBM) / C::kBM, p.nb_q - 1);
+        cl_q = p.scale * __ldg(p.dq_blk + static_cast<size_t>(bh) * p.nb_q + bq) * 1.4426950408889634f;
+        const float* dvr = p.dv_blk + static_cast<size_t>(bh) * p.nb_kv;
+        const int kt0 = p.k0 / C::kBN, kt1 = (p.k1 + C::kBN - 1) / C::kBN;
+        float mx = 0.0f;
+        for (int kt = kt0; kt < kt1; ++kt) mx = fmaxf(mx, __ldg(dvr + kt));
+        dv_out = mx;
+        dk_nxt = __ldg(p.dk_blk + static_cast<size_t>(bh) * p.nb_kv + kt0);
+        dv_nxt = __ldg(dvr + kt0);
+      }
+    }
     for (int j = 0; j < n_kv; ++j) {
       const int g = it * n_kv + j;
+      // e4m3: this tile's cl_j and V ratio; prefetch the next tile's descales
+      float clj = cl, lrj = 0.0f, inv_rj = 1.0f;
+      if constexpr (FP8) {
+        if (blk) {
+          const float dkj = dk_nxt, dvj = dv_nxt;
+          if (j + 1 < n_kv) {
+            const size_t nx = static_cast<size_t>(bh) * p.nb_kv + p.k0 / C::kBN + j + 1;
+            dk_nxt = __ldg(p.dk_blk + nx);
+            dv_nxt = __ldg(p.dv_blk + nx);
+          }
+          clj = cl_q * dkj;
+          if (dvj > 0.0f) {                  // an all-zero V block (descale 0) keeps r_j = 1
+            lrj = __log2f(dvj / dv_out);
+            inv_rj = dv_out / dvj;
+          }
+        }
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + t, g & 1, abort_flag, tmo, 11 + t));
       if (!ok) break;
       tc_fence_after();
@@ -463,13 +512,24 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld128_sync(tS, s);
           if (valid < C::kBN) mask_tail(s, valid);
         }
-        const float m_new = fmaxf(m_use, row_max128(s));
-        need = (m_new - m_use) * cl > C::kRescaleLog2;       // true on the first tile
-        if (need) {
-          alpha = ex2_approx((m_use - m_new) * cl);          // 0 when m_use = -inf
-          m_use = m_new;
+        if constexpr (FP8) {
+          const float m_new = fmaxf(m_use, clj * row_max128(s));
+          need = m_new - m_use > C::kRescaleLog2;            // true on the first tile
+          if (need) {
+            alpha = ex2_approx(m_use - m_new);               // 0 when m_use = -inf
+            m_use = m_new;
+          }
+          exp_pass<FP8, C::kEmuPer8>(s, clj, m_use - C::kPShift - lrj, pw, sum);
+          sum *= inv_rj;
+        } else {
+          const float m_new = fmaxf(m_use, row_max128(s));
+          need = (m_new - m_use) * cl > C::kRescaleLog2;     // true on the first tile
+          if (need) {
+            alpha = ex2_approx((m_use - m_new) * cl);        // 0 when m_use = -inf
+            m_use = m_new;
+          }
+          exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
         }
-        exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
       }
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
       if constexpr (!FP8) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));
@@ -500,7 +560,8 @@ __global__ void __launch_bounds__(384, 1)
       const bool store = grow < p.S_q;
       const size_t row_idx = static_cast<size_t>(bh) * p.S_q + grow;
       const size_t row_elem = row_idx * D;
-      const float lse_c = scale_eff * m_use + logf(l) - C::kPShift * 0.6931471805599453f;
+      const float lse_c = (FP8 ? m_use * 0.6931471805599453f : scale_eff * m_use) + logf(l) -
+                          C::kPShift * 0.6931471805599453f;
       // Accumulate mode (one ring step): (O, LSE) <- exact LSE merge of the running pair and
       // this range's partial, w = exp(lse - M) / L with M the larger LSE and L the weight sum.
       float w_old = 0.0f, w_new = 1.0f, lse_out = lse_c;
@@ -514,7 +575,7 @@ __global__ void __launch_bounds__(384, 1)
         w_new = ec / L;
         lse_out = M + logf(L);
       }
-      const float inv_l = dv / l * w_new;
+      const float inv_l = dv_out / l * w_new;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];

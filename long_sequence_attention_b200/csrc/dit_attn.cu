@@ -197,9 +197,17 @@ int noalloc_scratch(float** out) {
 
 namespace {
 
+// Per-block e4m3 descales (all three null for per-tensor scales).
+struct BlockScales {
+  const float* dq = nullptr;
+  const float* dk = nullptr;
+  const float* dv = nullptr;
+};
+
 int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S_q,
                     int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
-                    const float* descale_qkv, void* stream, bool accumulate) {
+                    const float* descale_qkv, void* stream, bool accumulate, const BlockScales& bs = BlockScales()) {
+  const bool blocks = bs.dq != nullptr || bs.dk != nullptr || bs.dv != nullptr;
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || S_q < 1 || S_kv < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (k0 < 0 || k1 < k0 || k1 > S_kv) return DIT_ERR_INVALID_ARG;
@@ -209,7 +217,12 @@ int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, floa
   if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
   const bool fp8 = dtype == DIT_FP8_E4M3;
   if (fp8 && D != 128) return DIT_ERR_UNSUPPORTED;
-  if (fp8 && descale_qkv == nullptr) return DIT_ERR_INVALID_ARG;
+  if (fp8 && !blocks && descale_qkv == nullptr) return DIT_ERR_INVALID_ARG;
+  if (blocks) {
+    if (!fp8 || bs.dq == nullptr || bs.dk == nullptr || bs.dv == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned(bs.dq, 4) || !aligned(bs.dk, 4) || !aligned(bs.dv, 4)) return DIT_ERR_MISALIGNED;
+    if (k0 % 128 != 0) return DIT_ERR_UNSUPPORTED;   // KV tiles must coincide with scale blocks
+  }
   if (static_cast<long long>(B) * H > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return DIT_ERR_MISALIGNED;
   if (lse != nullptr && !aligned(lse, 4)) return DIT_ERR_MISALIGNED;
@@ -242,6 +255,11 @@ int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, floa
   prm.lse = lse;
   prm.out_fp32 = out_dtype == DIT_FP32;
   prm.accumulate = accumulate ? 1 : 0;
+  prm.dq_blk = blocks ? bs.dq : nullptr;
+  prm.dk_blk = blocks ? bs.dk : nullptr;
+  prm.dv_blk = blocks ? bs.dv : nullptr;
+  prm.nb_q = (S_q + 127) / 128;
+  prm.nb_kv = (S_kv + 127) / 128;
   prm.timeout_ns = g_timeout_ns.load();
   if (fp8) return launch_attn<128, true>(q, k, v, prm, st);
   if (D == 64) return launch_attn<64, false>(q, k, v, prm, st);
@@ -265,6 +283,36 @@ int dit_attn_fwd_chunk_acc(const void* q, const void* k, const void* v, float* a
   if (acc_out == nullptr || acc_lse == nullptr) return DIT_ERR_INVALID_ARG;
   return attn_chunk_impl(q, k, v, acc_out, acc_lse, B, H, S_q, S_kv, D, k0, k1, scale, dtype, DIT_FP32,
                          descale_qkv, stream, true);
+}
+
+int dit_attn_fwd_fp8_blocks(const void* q8, const void* k8, const void* v8, const float* dq_blk, const float* dk_blk,
+                            const float* dv_blk, void* out, float* lse, int B, int H, int S_q, int S_kv, int D,
+                            int k0, int k1, float scale, int out_dtype, void* stream) {
+  if (dq_blk == nullptr || dk_blk == nullptr || dv_blk == nullptr) return DIT_ERR_INVALID_ARG;
+  BlockScales bs;
+  bs.dq = dq_blk;
+  bs.dk = dk_blk;
+  bs.dv = dv_blk;
+  return attn_chunk_impl(q8, k8, v8, out, lse, B, H, S_q, S_kv, D, k0, k1, scale, DIT_FP8_E4M3, out_dtype, nullptr,
+                         stream, false, bs);
+}
+
+int dit_quant_fp8_blocks(const void* x_bf16, void* x_fp8, float* descales, int B, int H, int S, int D,
+                         void* stream) {
+  if (x_bf16 == nullptr || x_fp8 == nullptr || descales == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || S < 1 || D < 8) return DIT_ERR_INVALID_ARG;
+  if (D % 8 != 0 || D > 128) return DIT_ERR_UNSUPPORTED;
+  if (!aligned(x_bf16, 16) || !aligned(x_fp8, 8) || !aligned(descales, 4)) return DIT_ERR_MISALIGNED;
+  const long long nblk = (S + 127) / 128;
+  const long long grid = static_cast<long long>(B) * H * nblk;
+  if (grid > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  const size_t n = static_cast<size_t>(B) * H * S * D;
+  if (overlaps(x_fp8, n, x_bf16, 2 * n) || overlaps(descales, static_cast<size_t>(grid) * 4, x_bf16, 2 * n) ||
+      overlaps(descales, static_cast<size_t>(grid) * 4, x_fp8, n))
+    return DIT_ERR_INVALID_ARG;
+  quant_e4m3_rows_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(x_bf16), S, D, static_cast<int>(nblk), static_cast<uint8_t*>(x_fp8), descales);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
 int dit_attn_acc_init(float* acc_out, float* acc_lse, int B, int H, int S, int D, void* stream) {

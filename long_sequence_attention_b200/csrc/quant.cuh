@@ -102,4 +102,57 @@ __global__ void __launch_bounds__(kQuantThreads) quant_e4m3_kernel(const uint16_
   }
 }
 
+// Per-block scales: one CTA per block of 128 consecutive rows of one (b, h) of a [B,H,S,D]
+// tensor (the last block of a head may be shorter).  The block (at most 128 x 128 bf16 =
+// 32 KB) is read once into registers, its absolute maximum reduced, and the codes written:
+// one HBM read and one write per element.  An all-zero block gets descale 0 (it holds only
+// zero codes; a consumer can tell it apart from a block whose maximum is 448) and codes of
+// x / 1, the per-tensor rule for an all-zero tensor.
+constexpr int kQuantBlockRows = 128;
+
+__global__ void __launch_bounds__(kQuantThreads) quant_e4m3_rows_kernel(const uint16_t* __restrict__ x, int S, int D,
+                                                                        int nblk, uint8_t* __restrict__ x8,
+                                                                        float* __restrict__ descales) {
+  __shared__ float red[kQuantThreads / 32];
+  const long long bh = blockIdx.x / nblk;
+  const int i = static_cast<int>(blockIdx.x - bh * nblk);
+  const int r0 = i * kQuantBlockRows;
+  const int rows = min(kQuantBlockRows, S - r0);
+  const long long base = (bh * S + r0) * static_cast<long long>(D);      // first element
+  const int nvec = rows * D / 8;                                         // D % 8 == 0
+  constexpr int kPer = kQuantBlockRows * 128 / 8 / kQuantThreads;        // vectors per thread (D <= 128)
+  uint4 a[kPer];
+  float m = 0.0f;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = threadIdx.x + k * kQuantThreads;
+    a[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (idx < nvec) a[k] = __ldg(reinterpret_cast<const uint4*>(x + base) + idx);
+    const uint32_t w[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      m = fmaxf(m, fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)));
+      m = fmaxf(m, fabsf(bf16_bits_to_float(w[e] >> 16)));
+    }
+  }
+  const float amax = block_max(m, red);
+  const float descale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  if (threadIdx.x == 0) descales[blockIdx.x] = (amax > 0.0f) ? descale : 0.0f;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int idx = threadIdx.x + k * kQuantThreads;
+    if (idx < nvec) {
+      const uint32_t w[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+      uint32_t packed[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        packed[h] = pack_e4m3x4(__fdiv_rn(bf16_bits_to_float(w[2 * h] & 0xFFFFu), descale),
+                                __fdiv_rn(bf16_bits_to_float(w[2 * h] >> 16), descale),
+                                __fdiv_rn(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), descale),
+                                __fdiv_rn(bf16_bits_to_float(w[2 * h + 1] >> 16), descale));
+      reinterpret_cast<uint2*>(x8 + base)[idx] = make_uint2(packed[0], packed[1]);
+    }
+  }
+}
+
 }  // namespace dit

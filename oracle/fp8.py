@@ -20,7 +20,9 @@ the FP8 layout or the scaling; the readings used here:
 * Per-block scale (a finer variant of the same scheme, not described by the pages): a
   [B,H,S,D] tensor is cut, per (b, h), into blocks of 128 consecutive rows (tokens), the
   last one ragged; each block is quantised exactly as a tensor of its own, with its own
-  descale.  Descales form a float32 [B,H,ceil(S/128)] array.
+  descale.  Descales form a float32 [B,H,ceil(S/128)] array.  An all-zero block records
+  descale 0 (its codes are those of x / 1, all zero): that tells it apart from a block whose
+  maximum is 448, and its dequantised values are zero either way.
 """
 
 from __future__ import annotations
@@ -108,6 +110,8 @@ def quantize_per_block(x: np.ndarray, block_rows: int = BLOCK_ROWS) -> Tuple[np.
             for i in range(nblk):
                 rows = slice(i * block_rows, min(S, (i + 1) * block_rows))
                 codes[b, h, rows], descales[b, h, i] = quantize_per_tensor(x32[b, h, rows])
+                if not np.any(x32[b, h, rows]):
+                    descales[b, h, i] = 0.0
     return codes, descales
 
 

@@ -409,7 +409,7 @@ def test_quantize_per_block_constructed_scales():
     x[1, 2, 128:256] = 0.0                                 # one all-zero block
     codes, ds = fp8.quantize_per_block(x.astype(np.float32))
     want_ds = np.broadcast_to(np.array([1.0, 2.0, 4.0], dtype=np.float32), (B, H, 3)).copy()
-    want_ds[1, 2, 1] = 1.0
+    want_ds[1, 2, 1] = 0.0                                 # all-zero block: descale 0
     assert ds.dtype == np.float32 and np.array_equal(ds, want_ds)
     want_codes = pattern_codes.copy()
     want_codes[1, 2, 128:256] = np.where(np.signbit(x[1, 2, 128:256]), 0x80, 0x00)
@@ -429,6 +429,11 @@ def test_quantize_per_block_is_per_tensor_on_each_block():
         for i, (a, b) in enumerate([(0, 128), (128, 256), (256, 300)]):
             c1, d1 = fp8.quantize_per_tensor(x[0, h, a:b])
             assert d1 == ds[0, h, i] and np.array_equal(c1, codes[0, h, a:b])
+    z = np.zeros((1, 1, 130, 8), dtype=np.float32)
+    z[0, 0, 0, 0] = -0.0
+    zc, zd = fp8.quantize_per_block(z)
+    assert np.array_equal(zd, np.zeros((1, 1, 2), dtype=np.float32))
+    assert np.array_equal(zc, fp8.quantize_per_tensor(z)[0])      # codes of x / 1
     cw, dw = fp8.quantize_per_block(x[:, :1], block_rows=300)
     ct, dt = fp8.quantize_per_tensor(x[:, :1])
     assert dw[0, 0, 0] == dt and np.array_equal(cw, ct)
