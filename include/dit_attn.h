@@ -109,6 +109,32 @@ int dit_attn_fwd_chunk_acc(const void* q, const void* k, const void* v, float* a
                            int dtype, const float* descale_qkv, void* stream);
 
 /*
+ * dit_attn_fwd_seg - dit_attn_fwd_chunk over all S keys (S_q = S_kv = S) for tensors stored in
+ * sequence segments: row r of head (b, h) at index ((r / seg) * B*H + b*H + h) * seg + r % seg,
+ * i.e. [S/seg, B, H, seg, D] (lse: [S/seg, B, H, seg]).  This is the layout in which the
+ * sequence-to-head all-to-all of the USP Ulysses dimension (xDiT overview page, section
+ * 3.2.2) delivers Q, K and V (segment p = the rows that came from rank p), and the layout
+ * its return all-to-all sends from, so neither side needs a re-layout copy.
+ *
+ *   seg       rows per segment; S % seg == 0; seg % 128 == 0 unless seg == S (seg == S is
+ *             the plain [B,H,S,D] layout), else DIT_ERR_UNSUPPORTED.
+ *   Other arguments as for dit_attn_fwd_chunk (out_dtype DIT_BF16 or DIT_FP32; E4M3 inputs
+ *   with per-tensor descales).
+ */
+int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                     int S, int D, int seg, float scale, int dtype, int out_dtype,
+                     const float* descale_qkv, void* stream);
+
+/*
+ * dit_swap01_chunks - dst[i1][i0] = src[i0][i1] for a [d0][d1] grid of chunks of chunk_bytes
+ * bytes each (the batch/peer transpose around a Ulysses all-to-all when B > 1).
+ *   src, dst  device buffers of d0 * d1 * chunk_bytes bytes, 16-byte aligned, not overlapping.
+ *   chunk_bytes a multiple of 16 (else DIT_ERR_UNSUPPORTED).
+ */
+int dit_swap01_chunks(const void* src, void* dst, long long d0, long long d1, long long chunk_bytes,
+                      void* stream);
+
+/*
  * dit_attn_acc_init - empty accumulator: acc_out = 0, acc_lse = -inf ([B,H,S,D] / [B,H,S] fp32).
  */
 int dit_attn_acc_init(float* acc_out, float* acc_lse, int B, int H, int S, int D, void* stream);

@@ -54,6 +54,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_selftest_wait_timeout.argtypes = [ull, vp]
     lib.dit_set_sm_reserve.argtypes = [i]
     lib.dit_quant_fp8_blocks.argtypes = [vp, vp, vp, i, i, i, i, vp]
+    lib.dit_attn_fwd_seg.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp]
+    lib.dit_swap01_chunks.argtypes = [vp, vp, ll, ll, ll, vp]
     lib.dit_attn_fwd_fp8_blocks.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
@@ -137,6 +139,17 @@ def dit_quant_fp8_workspace_bytes(n: int) -> int:
 def dit_quant_fp8(x_bf16, x_fp8, descale, n: int, workspace, workspace_bytes: int, stream=None) -> None:
     _check(lib.dit_quant_fp8(_ptr(x_bf16), _ptr(x_fp8), _ptr(descale), int(n), _ptr(workspace),
                              int(workspace_bytes), _stream(stream)), "dit_quant_fp8")
+
+
+def dit_attn_fwd_seg(q, k, v, out, lse, B: int, H: int, S: int, D: int, seg: int, scale: float,
+                     dtype: int = 0, out_dtype: int = 0, descale_qkv=None, stream=None) -> None:
+    _check(lib.dit_attn_fwd_seg(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D, seg, float(scale),
+                                dtype, out_dtype, _ptr(descale_qkv), _stream(stream)), "dit_attn_fwd_seg")
+
+
+def dit_swap01_chunks(src, dst, d0: int, d1: int, chunk_bytes: int, stream=None) -> None:
+    _check(lib.dit_swap01_chunks(_ptr(src), _ptr(dst), int(d0), int(d1), int(chunk_bytes), _stream(stream)),
+           "dit_swap01_chunks")
 
 
 def dit_quant_fp8_blocks(x_bf16, x_fp8, descales, B: int, H: int, S: int, D: int, stream=None) -> None:

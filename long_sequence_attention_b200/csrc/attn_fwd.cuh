@@ -68,6 +68,10 @@ struct AttnParams {
   const float* dk_blk;
   const float* dv_blk;
   int nb_q, nb_kv;
+  // Sequence segments: row r of head bh lives at ((r / seg) * B*H + bh) * seg + r % seg (the
+  // layout [S/seg, B*H, seg, D] that an all-to-all over the sequence leaves behind).
+  // seg = S is the plain [B, H, S, D] layout.
+  int seg_q, seg_kv;
   unsigned long long timeout_ns;
 };
 
@@ -291,8 +295,8 @@ __global__ void __launch_bounds__(384, 1)
         mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_3d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
-                        q0 + t * C::kBM, bh);
+            tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
+                        (q0 + t * C::kBM) % p.seg_q, bh, (q0 + t * C::kBM) / p.seg_q);
         q_issued = it + 1;
         for (int j = 0; j < n_kv; ++j) {
           const int g = it * n_kv + j;
@@ -303,8 +307,8 @@ __global__ void __launch_bounds__(384, 1)
             break;
           mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
           for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_3d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
-                        b * C::kBoxInner, kv_row, bh);
+            tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
+                        b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
           k_issued = g + 1;
           const int vs = g % C::kVStages;
           if (g >= C::kVStages &&
@@ -312,8 +316,8 @@ __global__ void __launch_bounds__(384, 1)
             break;
           mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
           for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_3d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
-                        b * C::kBoxInner, kv_row, bh);
+            tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
+                        b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
           v_issued = g + 1;
         }
       }
@@ -558,7 +562,8 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const int grow = q_start + t * C::kBM + row;
       const bool store = grow < p.S_q;
-      const size_t row_idx = static_cast<size_t>(bh) * p.S_q + grow;
+      const size_t row_idx =
+          (static_cast<size_t>(grow / p.seg_q) * p.B * p.H + bh) * p.seg_q + grow % p.seg_q;
       const size_t row_elem = row_idx * D;
       const float lse_c = (FP8 ? m_use * 0.6931471805599453f : scale_eff * m_use) + logf(l) -
                           C::kPShift * 0.6931471805599453f;

@@ -13,6 +13,7 @@
 #include "attn_fwd.cuh"
 #include "merge.cuh"
 #include "quant.cuh"
+#include "layout.cuh"
 
 namespace {
 
@@ -51,15 +52,21 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 
 // 3-D tiled map over a [B*H, S, D] tensor: box = (128 bytes of D, 128 rows, 1 head),
 // 128-byte swizzle, zero fill out of bounds (rows past S read as zeros, per head).
-int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH) {
+// 4-D map (D, seg, BH, S / seg) of a tensor whose rows are stored in sequence segments:
+// row r of head bh at ((r / seg) * BH + bh) * seg + r % seg.  seg = S is the plain
+// [BH, S, D] layout.  Box: 128 bytes x 128 rows, 128-byte swizzle; rows past a segment or
+// past the last segment read as zero.
+int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH, int seg) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return DIT_ERR_CUDA;
   const cuuint64_t elem = fp8 ? 1 : 2;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * elem, static_cast<cuuint64_t>(S) * D * elem};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), 128, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  const cuuint64_t n_seg = static_cast<cuuint64_t>(S / seg);
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(seg), static_cast<cuuint64_t>(BH), n_seg};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * elem, static_cast<cuuint64_t>(seg) * D * elem,
+                           static_cast<cuuint64_t>(BH) * seg * D * elem};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / elem), 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
                          const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -124,9 +131,9 @@ int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p
   if (rc != DIT_OK) return rc;
   CUtensorMap tq, tk, tv;
   const int BH = prm.B * prm.H;
-  if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH)) != DIT_OK) return rc;
-  if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
-  if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH)) != DIT_OK) return rc;
+  if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH, prm.seg_q)) != DIT_OK) return rc;
+  if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
+  if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
   AttnParams pr = prm;
   pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
   pr.n_units = pr.n_qblk * prm.H * prm.B;
@@ -206,8 +213,15 @@ struct BlockScales {
 
 int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S_q,
                     int S_kv, int D, int k0, int k1, float scale, int dtype, int out_dtype,
-                    const float* descale_qkv, void* stream, bool accumulate, const BlockScales& bs = BlockScales()) {
+                    const float* descale_qkv, void* stream, bool accumulate, const BlockScales& bs = BlockScales(),
+                    int seg = 0) {
   const bool blocks = bs.dq != nullptr || bs.dk != nullptr || bs.dv != nullptr;
+  // seg > 0: q, k, v, out and lse in sequence segments of seg rows (S_q == S_kv, k0 = 0)
+  if (seg < 0) return DIT_ERR_INVALID_ARG;
+  if (seg > 0) {
+    if (S_q != S_kv || k0 != 0 || k1 != S_kv || S_q % seg != 0) return DIT_ERR_INVALID_ARG;
+    if (seg != S_q && seg % 128 != 0) return DIT_ERR_UNSUPPORTED;   // tiles must not straddle segments
+  }
   if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || S_q < 1 || S_kv < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (k0 < 0 || k1 < k0 || k1 > S_kv) return DIT_ERR_INVALID_ARG;
@@ -260,6 +274,8 @@ int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, floa
   prm.dv_blk = blocks ? bs.dv : nullptr;
   prm.nb_q = (S_q + 127) / 128;
   prm.nb_kv = (S_kv + 127) / 128;
+  prm.seg_q = seg > 0 ? seg : S_q;
+  prm.seg_kv = seg > 0 ? seg : S_kv;
   prm.timeout_ns = g_timeout_ns.load();
   if (fp8) return launch_attn<128, true>(q, k, v, prm, st);
   if (D == 64) return launch_attn<64, false>(q, k, v, prm, st);
@@ -295,6 +311,28 @@ int dit_attn_fwd_fp8_blocks(const void* q8, const void* k8, const void* v8, cons
   bs.dv = dv_blk;
   return attn_chunk_impl(q8, k8, v8, out, lse, B, H, S_q, S_kv, D, k0, k1, scale, DIT_FP8_E4M3, out_dtype, nullptr,
                          stream, false, bs);
+}
+
+int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int S,
+                     int D, int seg, float scale, int dtype, int out_dtype, const float* descale_qkv,
+                     void* stream) {
+  if (seg < 1) return DIT_ERR_INVALID_ARG;
+  return attn_chunk_impl(q, k, v, out, lse, B, H, S, S, D, 0, S, scale, dtype, out_dtype, descale_qkv, stream,
+                         false, BlockScales(), seg);
+}
+
+int dit_swap01_chunks(const void* src, void* dst, long long d0, long long d1, long long chunk_bytes,
+                      void* stream) {
+  if (src == nullptr || dst == nullptr || d0 < 1 || d1 < 1 || chunk_bytes < 16) return DIT_ERR_INVALID_ARG;
+  if (chunk_bytes % 16 != 0) return DIT_ERR_UNSUPPORTED;
+  if (!aligned(src, 16) || !aligned(dst, 16)) return DIT_ERR_MISALIGNED;
+  if (d0 > (1LL << 40) / d1 || d0 * d1 > (1LL << 48) / chunk_bytes) return DIT_ERR_INVALID_ARG;
+  const long long bytes = d0 * d1 * chunk_bytes;
+  if (overlaps(dst, static_cast<size_t>(bytes), src, static_cast<size_t>(bytes))) return DIT_ERR_INVALID_ARG;
+  const long long vecs = bytes / 16;
+  swap01_chunks_kernel<<<grid_for(vecs, 256, 148 * 8), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), d0, d1, chunk_bytes / 16);
+  return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
 int dit_quant_fp8_blocks(const void* x_bf16, void* x_fp8, float* descales, int B, int H, int S, int D,
