@@ -15,6 +15,8 @@ Contents
                    per-tensor absmax quantisation, written from the format definition.
 ``brute``          an independent triple-loop C implementation in ``long double`` for
                    tiny shapes (``brute_attention.c``), used to pin ``attention``.
+``neighborhood``   3-D neighborhood attention on a T x Y x X token grid (the NATTEN
+                   na3d operation): clamped fixed-size windows, explicit softmax, fp64.
 
 Parity status: every function here is pinned by ``tests/test_oracle.py`` (brute force,
 closed forms, invariants, a library cross-check and planted-mistake checks).
@@ -22,3 +24,4 @@ closed forms, invariants, a library cross-check and planted-mistake checks).
 
 from .attn import attention, softmax_rows, merge, NEG_INF  # noqa: F401
 from . import fp8  # noqa: F401
+from . import neighborhood  # noqa: F401

@@ -444,3 +444,92 @@ def test_quantize_per_block_is_per_tensor_on_each_block():
     def rel(a):
         return np.linalg.norm(a[0, 0] - x[0, 0]) / np.linalg.norm(x[0, 0])
     assert rel(fp8.dequantize_per_block(codes, ds)) < 0.05 and rel(fp8.dequantize(ct2, dt2)) > 0.2
+
+
+# ------------------------------------------------------------------ neighborhood attention
+from oracle import neighborhood as nbh  # noqa: E402
+
+
+def test_window_start_is_the_nearest_k_positions():
+    """The clamped window equals the K positions nearest to i (by brute force over the line;
+    for odd K there is never a tie at the window's edge)."""
+    for L in range(1, 13):
+        for K in range(1, L + 1, 2):
+            for i in range(L):
+                order = sorted(range(L), key=lambda j: (abs(j - i), j))
+                near = sorted(order[:K])
+                assert abs(order[K - 1] - i) < abs(order[K] - i) if K < L else True
+                st = nbh.window_start(i, K, L)
+                assert near == list(range(st, st + K)), (L, K, i)
+    with pytest.raises(ValueError):
+        nbh.window_start(0, 4, 10)
+    with pytest.raises(ValueError):
+        nbh.window_start(0, 5, 3)
+
+
+def _na_loops(q, k, v, grid, kernel, scale):
+    """Pure-Python loops: key j is a neighbour of query i when, in every dimension, j's
+    coordinate is among the K coordinates nearest to i's (the definition above, written
+    without window_start)."""
+    import math
+    T, Y, X = grid
+    B, H, S, D = q.shape
+
+    def near(i, K, L):
+        return set(sorted(range(L), key=lambda j: (abs(j - i), j))[:K])
+
+    out = np.zeros((B, H, S, D))
+    lse = np.zeros((B, H, S))
+    for b in range(B):
+        for h in range(H):
+            for s in range(S):
+                t, y, x = s // (Y * X), (s // X) % Y, s % X
+                nt, ny, nx = near(t, kernel[0], T), near(y, kernel[1], Y), near(x, kernel[2], X)
+                keys = [j for j in range(S) if j // (Y * X) in nt and (j // X) % Y in ny and j % X in nx]
+                xs = [scale * sum(float(q[b, h, s, d]) * float(k[b, h, j, d]) for d in range(D)) for j in keys]
+                m = max(xs)
+                es = [math.exp(a - m) for a in xs]
+                den = sum(es)
+                for d in range(D):
+                    out[b, h, s, d] = sum(e * float(v[b, h, j, d]) for e, j in zip(es, keys)) / den
+                lse[b, h, s] = m + math.log(den)
+    return out, lse
+
+
+@pytest.mark.parametrize("grid,kernel", [((2, 3, 4), (1, 3, 3)), ((3, 4, 5), (3, 3, 1)), ((1, 5, 6), (1, 3, 5)),
+                                         ((4, 2, 3), (3, 1, 3))])
+def test_neighborhood_matches_loops(grid, kernel):
+    S = int(np.prod(grid))
+    q, k, v = (make_tensor((1, 2, S, 3), seed) for seed in (21, 22, 23))
+    o, l = nbh.neighborhood_attention_3d(q, k, v, grid, kernel, 0.7)
+    ro, rl = _na_loops(q, k, v, grid, kernel, 0.7)
+    assert np.allclose(o, ro, rtol=0, atol=1e-12) and np.allclose(l, rl, rtol=0, atol=1e-12)
+
+
+def test_neighborhood_full_window_is_full_attention():
+    grid = (3, 5, 7)
+    q, k, v = (make_tensor((2, 1, 105, 8), seed) for seed in (31, 32, 33))
+    o, l = nbh.neighborhood_attention_3d(q, k, v, grid, grid, 0.3)
+    ro, rl = oracle.attention(q, k, v, 0.3)
+    assert np.allclose(o, ro, rtol=0, atol=1e-12) and np.allclose(l, rl, rtol=0, atol=1e-12)
+
+
+def test_neighborhood_unit_window_is_self():
+    grid = (2, 3, 4)
+    q, k, v = (make_tensor((1, 2, 24, 4), seed) for seed in (41, 42, 43))
+    o, l = nbh.neighborhood_attention_3d(q, k, v, grid, (1, 1, 1), 0.5)
+    assert np.array_equal(o, v.astype(np.float64))
+    assert np.allclose(l, 0.5 * np.einsum("bhsd,bhsd->bhs", q.astype(np.float64), k.astype(np.float64)),
+                       rtol=0, atol=1e-12)
+
+
+def test_neighborhood_rows_subset_and_counts():
+    grid, kernel = (5, 6, 7), (3, 5, 3)
+    q, k, v = (make_tensor((1, 1, 210, 4), seed) for seed in (51, 52, 53))
+    o, l = nbh.neighborhood_attention_3d(q, k, v, grid, kernel, 0.4)
+    rows = [0, 6, 41, 209, 100]
+    os_, ls = nbh.neighborhood_attention_3d(q, k, v, grid, kernel, 0.4, rows=rows)
+    assert np.array_equal(os_, o[:, :, rows]) and np.array_equal(ls, l[:, :, rows])
+    for s in range(210):
+        idx = nbh.neighbor_index(grid, kernel, s)
+        assert len(set(idx.tolist())) == 45 and s in idx
