@@ -126,6 +126,24 @@ int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, flo
                      const float* descale_qkv, void* stream);
 
 /*
+ * dit_na3d_fwd - 3-D neighborhood attention on a T x Y x X token grid (the operation NATTEN
+ * calls na3d; the LTX notes page, section 5, reports it as the hot spot of a video decoder).
+ * Token s = (t * Y + y) * X + x of each (b, h) attends only to the keys of its neighborhood:
+ * along each dimension of length L with odd window K, the K positions starting at
+ * clamp(i - K/2, 0, L - K) (fixed size, shifted inward at the borders; dilation 1,
+ * non-causal); the neighborhood is the product of the three windows.
+ *     out_s = sum_{j in N(s)} softmax_j(scale * q_s . k_j) v_j,
+ *     lse_s = log sum_{j in N(s)} exp(scale * q_s . k_j).
+ *
+ *   q, k, v   [B,H,T*Y*X,D] bf16;  out [B,H,T*Y*X,D] bf16;  lse [B,H,T*Y*X] fp32 or NULL.
+ *   Kt, Ky, Kx odd, 1 <= K <= the grid dimension, else DIT_ERR_INVALID_ARG.  D = 64 or 128.
+ *   The kernel visits only the 128-token bricks (4 x 4 x 8 in t, y, x) that some window of
+ *   its queries touches and masks, per query, the keys outside that query's window.
+ */
+int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                 int T, int Y, int X, int D, int Kt, int Ky, int Kx, float scale, void* stream);
+
+/*
  * dit_swap01_chunks - dst[i1][i0] = src[i0][i1] for a [d0][d1] grid of chunks of chunk_bytes
  * bytes each (the batch/peer transpose around a Ulysses all-to-all when B > 1).
  *   src, dst  device buffers of d0 * d1 * chunk_bytes bytes, 16-byte aligned, not overlapping.

@@ -56,6 +56,7 @@ def _load() -> ctypes.CDLL:
     lib.dit_quant_fp8_blocks.argtypes = [vp, vp, vp, i, i, i, i, vp]
     lib.dit_attn_fwd_seg.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp]
     lib.dit_swap01_chunks.argtypes = [vp, vp, ll, ll, ll, vp]
+    lib.dit_na3d_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp]
     lib.dit_attn_fwd_fp8_blocks.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
@@ -145,6 +146,25 @@ def dit_attn_fwd_seg(q, k, v, out, lse, B: int, H: int, S: int, D: int, seg: int
                      dtype: int = 0, out_dtype: int = 0, descale_qkv=None, stream=None) -> None:
     _check(lib.dit_attn_fwd_seg(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D, seg, float(scale),
                                 dtype, out_dtype, _ptr(descale_qkv), _stream(stream)), "dit_attn_fwd_seg")
+
+
+def dit_na3d_fwd(q, k, v, out, lse, B: int, H: int, T: int, Y: int, X: int, D: int, Kt: int, Ky: int, Kx: int,
+                 scale: float, stream=None) -> None:
+    _check(lib.dit_na3d_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, T, Y, X, D, Kt, Ky, Kx,
+                            float(scale), _stream(stream)), "dit_na3d_fwd")
+
+
+def neighborhood_attention(q, k, v, grid, kernel, scale: Optional[float] = None, with_lse: bool = True,
+                           stream=None):
+    """(out bf16, lse fp32 or None) of 3-D neighborhood attention; q, k, v [B,H,T*Y*X,D] bf16,
+    grid = (T, Y, X), kernel = (Kt, Ky, Kx)."""
+    import torch
+    B, H, S, D = _dims(q)
+    scale = (1.0 / D ** 0.5) if scale is None else scale
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device) if with_lse else None
+    dit_na3d_fwd(q, k, v, out, lse, B, H, *grid, D, *kernel, scale, stream)
+    return out, lse
 
 
 def dit_swap01_chunks(src, dst, d0: int, d1: int, chunk_bytes: int, stream=None) -> None:

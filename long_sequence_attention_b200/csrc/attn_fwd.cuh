@@ -72,8 +72,89 @@ struct AttnParams {
   // layout [S/seg, B*H, seg, D] that an all-to-all over the sequence leaves behind).
   // seg = S is the plain [B, H, S, D] layout.
   int seg_q, seg_kv;
+  // Neighborhood attention (the NA instantiation only): T x Y x X token grid, odd window
+  // sizes, and the unit grid (Q bricks along t, brick pairs along y, bricks along x).
+  int na_T, na_Y, na_X;
+  int na_Kt, na_Ky, na_Kx;
+  int na_nbt, na_nby2, na_nbx;
   unsigned long long timeout_ns;
 };
+
+// ---------------------------------------------------------------------------------------
+// Neighborhood attention geometry (the operation NATTEN calls na3d; the LTX notes page,
+// section 5, reports it as the decoder's hot spot).  The neighborhood of a query at
+// position i along a dimension of length L is the K positions starting at
+// clamp(i - K/2, 0, L - K); the 3-D neighborhood is the product over (t, y, x).
+// A 128-row tile is a brick of kNaBt x kNaBy x kNaBx tokens, loaded by one 5-D TMA box
+// (x fastest), so tile row c is the token (c / 32, (c / 8) % 4, c % 8) of the brick.  A unit
+// is two bricks stacked along y; it visits every KV brick that the windows of its queries
+// touch (the union of windows, rounded out to bricks), and each row masks the keys outside
+// its own window.
+// ---------------------------------------------------------------------------------------
+constexpr int kNaBt = 4, kNaBy = 4, kNaBx = 8;
+
+__device__ __forceinline__ int na_wstart(int i, int K, int L) { return min(max(i - K / 2, 0), L - K); }
+
+struct NaUnit {
+  int bh;
+  int qt, qy, qx;        // token origin of Q brick 0 (brick 1 is kNaBy further along y)
+  int bt0, by0, bx0;     // first KV brick (in bricks)
+  int nt, ny, nx;        // KV bricks along t, y, x
+  __device__ __forceinline__ int n() const { return nt * ny * nx; }
+  // token origin of KV tile j (x fastest, then y, then t)
+  __device__ __forceinline__ void kv_origin(int j, int& t, int& y, int& x) const {
+    const int jx = j % nx, jy = (j / nx) % ny, jt = j / (nx * ny);
+    t = (bt0 + jt) * kNaBt;
+    y = (by0 + jy) * kNaBy;
+    x = (bx0 + jx) * kNaBx;
+  }
+};
+
+// KV bricks covering the windows of the queries [a, min(a + ext, L)) along one dimension.
+__device__ __forceinline__ void na_span(int a, int ext, int K, int L, int b, int& first, int& count) {
+  const int last = min(a + ext, L) - 1;
+  const int lo = na_wstart(a, K, L), hi = na_wstart(last, K, L) + K;
+  first = lo / b;
+  count = (hi + b - 1) / b - first;
+}
+
+__device__ __forceinline__ NaUnit na_unit(const AttnParams& p, int u) {
+  NaUnit w;
+  const int per_bh = p.na_nbt * p.na_nby2 * p.na_nbx;
+  w.bh = u / per_bh;
+  const int r = u - w.bh * per_bh;
+  const int ix = r % p.na_nbx, iy = (r / p.na_nbx) % p.na_nby2, it = r / (p.na_nbx * p.na_nby2);
+  w.qt = it * kNaBt;
+  w.qy = iy * 2 * kNaBy;
+  w.qx = ix * kNaBx;
+  na_span(w.qt, kNaBt, p.na_Kt, p.na_T, kNaBt, w.bt0, w.nt);
+  na_span(w.qy, 2 * kNaBy, p.na_Ky, p.na_Y, kNaBy, w.by0, w.ny);
+  na_span(w.qx, kNaBx, p.na_Kx, p.na_X, kNaBx, w.bx0, w.nx);
+  return w;
+}
+
+// 128-bit key mask of one query row for a KV brick at token origin (ot, oy, ox): bit c set
+// when key c of the brick lies in the row's window [ws, ws + K) along every dimension.
+// Word w covers brick plane t = w (4 y-rows of 8 x-bits).
+__device__ __forceinline__ void na_row_mask(int wt, int wy, int wx, int Kt, int Ky, int Kx, int ot, int oy, int ox,
+                                            uint32_t (&mw)[4]) {
+  const int lx = min(max(wx - ox, 0), kNaBx), hx = min(max(wx + Kx - ox, 0), kNaBx);
+  const int ly = min(max(wy - oy, 0), kNaBy), hy = min(max(wy + Ky - oy, 0), kNaBy);
+  const int lt = wt - ot, ht = wt + Kt - ot;
+  const uint32_t xbits = ((1u << hx) - 1u) & ~((1u << lx) - 1u);          // <= 8 bits
+  uint32_t ymul = 0u;
+#pragma unroll
+  for (int cy = 0; cy < kNaBy; ++cy) ymul |= (cy >= ly && cy < hy) ? (1u << (8 * cy)) : 0u;
+  const uint32_t plane = xbits * ymul;                                     // no carries: xbits < 256
+#pragma unroll
+  for (int ct = 0; ct < kNaBt; ++ct) mw[ct] = (ct >= lt && ct < ht) ? plane : 0u;
+}
+
+__device__ __forceinline__ void apply_mask128(uint32_t (&s)[128], const uint32_t (&mw)[4]) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xFF800000u;
+}
 
 // exp2 on the FMA pipe for x <= 2^7: x = n + f with n = rint(x), f in [-1/2, 1/2];
 // 2^f by a degree-3 polynomial (minimax in relative error, max 7.5e-5; coefficients from
@@ -221,7 +302,7 @@ __device__ __forceinline__ void exp_pass(const uint32_t (&s)[128], float cl, flo
   sum = lo + hi;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool NA = false>
 __global__ void __launch_bounds__(384, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -287,39 +368,65 @@ __global__ void __launch_bounds__(384, 1)
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       int k_issued = 0, v_issued = 0, q_issued = 0;   // running counts over all units
+      int g0 = 0;                                      // running KV tile count at unit start
       bool ok = true;
       for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
-        const int bh = unit_bh(u), q0 = unit_q0(u);
+        NaUnit w;
+        int bh, q0, nkv;
+        if constexpr (NA) {
+          w = na_unit(p, u);
+          bh = w.bh; q0 = 0; nkv = w.n();
+        } else {
+          bh = unit_bh(u); q0 = unit_q0(u); nkv = n_kv;
+        }
         // Q of this unit may overwrite the previous unit's only after its last S MMA.
         if (it > 0 && !(ok = mbar_wait(bar_q_empty, (it - 1) & 1, abort_flag, tmo, 0))) break;
         mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
-          for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
-                        (q0 + t * C::kBM) % p.seg_q, bh, (q0 + t * C::kBM) / p.seg_q);
+          for (int b = 0; b < C::kNBlk; ++b) {
+            if constexpr (NA)
+              tma_load_5d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner, w.qx,
+                          w.qy + t * kNaBy, w.qt, bh);
+            else
+              tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
+                          (q0 + t * C::kBM) % p.seg_q, bh, (q0 + t * C::kBM) / p.seg_q);
+          }
         q_issued = it + 1;
-        for (int j = 0; j < n_kv; ++j) {
-          const int g = it * n_kv + j;
+        for (int j = 0; j < nkv; ++j) {
+          const int g = g0 + j;
           const int kv_row = p.k0 + j * C::kBN;
+          int ot = 0, oy = 0, ox = 0;
+          if constexpr (NA) w.kv_origin(j, ot, oy, ox);
           const int ks = g % C::kKStages;
           if (g >= C::kKStages &&
               !(ok = mbar_wait(bar_k_empty + ks, ((g / C::kKStages) + 1) & 1, abort_flag, tmo, 1)))
             break;
           mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
-          for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
-                        b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
+          for (int b = 0; b < C::kNBlk; ++b) {
+            if constexpr (NA)
+              tma_load_5d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks, b * C::kBoxInner,
+                          ox, oy, ot, bh);
+            else
+              tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
+                          b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
+          }
           k_issued = g + 1;
           const int vs = g % C::kVStages;
           if (g >= C::kVStages &&
               !(ok = mbar_wait(bar_v_empty + vs, ((g / C::kVStages) + 1) & 1, abort_flag, tmo, 2)))
             break;
           mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
-          for (int b = 0; b < C::kNBlk; ++b)
-            tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
-                        b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
+          for (int b = 0; b < C::kNBlk; ++b) {
+            if constexpr (NA)
+              tma_load_5d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs, b * C::kBoxInner,
+                          ox, oy, ot, bh);
+            else
+              tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
+                          b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
+          }
           v_issued = g + 1;
         }
+        g0 += nkv;
       }
       // Drain: the last load armed on every stage must land before the CTA may exit
       // (a no-op in a healthy run, where the consumers already waited for all of them).
@@ -374,11 +481,14 @@ __global__ void __launch_bounds__(384, 1)
       };
 
       bool ok = true;
+      int g0 = 0;                                      // running KV tile count at unit start
       for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+        int nkv;
+        if constexpr (NA) nkv = na_unit(p, u).n();
+        else nkv = n_kv;
         if (!(ok = mbar_wait(bar_q_full, it & 1, abort_flag, tmo, 3))) break;
         tc_fence_after();
-        const int g0 = it * n_kv;
-        for (int j = 0; ok && j < n_kv; ++j) {
+        for (int j = 0; ok && j < nkv; ++j) {
           const int g = g0 + j;
           const int ks = g % C::kKStages;
           if (!(ok = mbar_wait(bar_k_full + ks, (g / C::kKStages) & 1, abort_flag, tmo, 4))) break;
@@ -404,21 +514,22 @@ __global__ void __launch_bounds__(384, 1)
         }
         if (!ok) break;
         tc_commit(bar_q_empty);                    // every S MMA of this unit is issued
-        const int gl = g0 + n_kv - 1, vs = gl % C::kVStages;
+        const int gl = g0 + nkv - 1, vs = gl % C::kVStages;
         ok = mbar_wait(bar_v_full + vs, (gl / C::kVStages) & 1, abort_flag, tmo, 8);
         if (ok) ok = mbar_wait(bar_p_full + 0, gl & 1, abort_flag, tmo, 9);
         if (ok) {
           tc_fence_after();
-          issue_pv(0, vs, n_kv > 1);
+          issue_pv(0, vs, nkv > 1);
           tc_commit(bar_o_final + 0);
           ok = mbar_wait(bar_p_full + 1, gl & 1, abort_flag, tmo, 10);
         }
         if (ok) {
           tc_fence_after();
-          issue_pv(1, vs, n_kv > 1);
+          issue_pv(1, vs, nkv > 1);
           tc_commit(bar_o_final + 1);
           tc_commit(bar_v_empty + vs);
         }
+        g0 += nkv;
       }
       // Every MMA this thread issued must finish before TMEM is released.
       tc_commit(bar_drain);
@@ -452,8 +563,23 @@ __global__ void __launch_bounds__(384, 1)
     const float cl = scale_eff * 1.4426950408889634f;          // log2 units per raw score
     bool ok = true;
 
+    int g0 = 0;                                                // running KV tile count at unit start
     for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
-    const int bh = unit_bh(u), q_start = unit_q0(u);
+    NaUnit w;
+    int bh, q_start, nkv;
+    int qt = 0, qy = 0, qx = 0, wt = 0, wy = 0, wx = 0;       // NA: this row's token and window starts
+    if constexpr (NA) {
+      w = na_unit(p, u);
+      bh = w.bh; q_start = 0; nkv = w.n();
+      qt = w.qt + row / (kNaBy * kNaBx);
+      qy = w.qy + t * kNaBy + (row / kNaBx) % kNaBy;
+      qx = w.qx + row % kNaBx;
+      wt = na_wstart(qt, p.na_Kt, p.na_T);
+      wy = na_wstart(qy, p.na_Ky, p.na_Y);
+      wx = na_wstart(qx, p.na_Kx, p.na_X);
+    } else {
+      bh = unit_bh(u); q_start = unit_q0(u); nkv = n_kv;
+    }
     float m_use = -INFINITY;             // running (lazy) max: raw units (bf16), log2 units (e4m3)
     float l = 0.0f;
     float cl_q = cl, dv_out = dv;        // per unit and Q tile (e4m3 per-block scales)
@@ -471,14 +597,14 @@ __global__ void __launch_bounds__(384, 1)
         dv_nxt = __ldg(dvr + kt0);
       }
     }
-    for (int j = 0; j < n_kv; ++j) {
-      const int g = it * n_kv + j;
+    for (int j = 0; j < nkv; ++j) {
+      const int g = g0 + j;
       // e4m3: this tile's cl_j and V ratio; prefetch the next tile's descales
       float clj = cl, lrj = 0.0f, inv_rj = 1.0f;
       if constexpr (FP8) {
         if (blk) {
           const float dkj = dk_nxt, dvj = dv_nxt;
-          if (j + 1 < n_kv) {
+          if (j + 1 < nkv) {
             const size_t nx = static_cast<size_t>(bh) * p.nb_kv + p.k0 / C::kBN + j + 1;
             dk_nxt = __ldg(p.dk_blk + nx);
             dv_nxt = __ldg(p.dv_blk + nx);
@@ -496,7 +622,17 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
       const int valid = p.k1 - (p.k0 + j * C::kBN);
-      if (valid < C::kBN) mask_tail(s, valid);
+      uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
+      bool part = false;                   // NA: some key of this tile lies outside the row's window
+      if constexpr (NA) {
+        int ot, oy, ox;
+        w.kv_origin(j, ot, oy, ox);
+        na_row_mask(wt, wy, wx, p.na_Kt, p.na_Ky, p.na_Kx, ot, oy, ox, mw);
+        part = (mw[0] & mw[1] & mw[2] & mw[3]) != ~0u;
+        if (part) apply_mask128(s, mw);
+      } else {
+        if (valid < C::kBN) mask_tail(s, valid);
+      }
       // Speculative pass (bf16): exponentiate with the running max m_use and keep the result
       // when the row sum shows that no p exceeds the lazy-rescale bound (every p <= sum <=
       // kSumBound), the usual case after the first tile.  Otherwise (first tile, a row max
@@ -506,7 +642,8 @@ __global__ void __launch_bounds__(384, 1)
       float sum;
       float alpha = 1.0f;
       bool need = false;
-      bool slow = (j == 0) || !C::kSpeculative;
+      // (NA: a row whose window has missed every tile so far has no max yet: exact route)
+      bool slow = (j == 0) || !C::kSpeculative || (NA && __any_sync(0xffffffffu, m_use == -INFINITY));
       if (!slow) {
         exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
         slow = __any_sync(0xffffffffu, !(sum <= C::kSumBound));
@@ -514,7 +651,11 @@ __global__ void __launch_bounds__(384, 1)
       if (slow) {
         if (j > 0 && C::kSpeculative) {
           tmem_ld128_sync(tS, s);
-          if (valid < C::kBN) mask_tail(s, valid);
+          if constexpr (NA) {
+            if (part) apply_mask128(s, mw);
+          } else {
+            if (valid < C::kBN) mask_tail(s, valid);
+          }
         }
         if constexpr (FP8) {
           const float m_new = fmaxf(m_use, clj * row_max128(s));
@@ -532,7 +673,9 @@ __global__ void __launch_bounds__(384, 1)
             alpha = ex2_approx((m_use - m_new) * cl);        // 0 when m_use = -inf
             m_use = m_new;
           }
-          exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
+          // (a row with no key in its window yet keeps m_use = -inf: exponents of -inf, p = 0)
+          const float mc = (NA && m_use == -INFINITY) ? 0.0f : m_use * cl;
+          exp_pass<FP8, C::kEmuPer8>(s, cl, mc - C::kPShift, pw, sum);
         }
       }
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
@@ -556,14 +699,22 @@ __global__ void __launch_bounds__(384, 1)
       if (lane == 0) mbar_arrive(bar_p_full + t);
     }
 
+    g0 += nkv;
+
     // ---------------------------------------------------------------- epilogue
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar_o_final + t, it & 1, abort_flag, tmo, 13 + t));
     if (ok) {
       tc_fence_after();
       const int grow = q_start + t * C::kBM + row;
-      const bool store = grow < p.S_q;
-      const size_t row_idx =
-          (static_cast<size_t>(grow / p.seg_q) * p.B * p.H + bh) * p.seg_q + grow % p.seg_q;
+      bool store;
+      size_t row_idx;
+      if constexpr (NA) {
+        store = qt < p.na_T && qy < p.na_Y && qx < p.na_X;
+        row_idx = static_cast<size_t>(bh) * p.S_q + (static_cast<size_t>(qt) * p.na_Y + qy) * p.na_X + qx;
+      } else {
+        store = grow < p.S_q;
+        row_idx = (static_cast<size_t>(grow / p.seg_q) * p.B * p.H + bh) * p.seg_q + grow % p.seg_q;
+      }
       const size_t row_elem = row_idx * D;
       const float lse_c = (FP8 ? m_use * 0.6931471805599453f : scale_eff * m_use) + logf(l) -
                           C::kPShift * 0.6931471805599453f;

@@ -73,6 +73,26 @@ int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH, in
   return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
 }
 
+// 5-D map (D, X, Y, T, BH) of a bf16 [BH, T*Y*X, D] tensor on a T x Y x X token grid for
+// the neighborhood-attention kernel.  Box: 128 bytes x an 8 x 4 x 4 (x, y, t) brick of
+// tokens = 128 rows, 128-byte swizzle; tokens past the grid read as zero.
+int make_map_na(CUtensorMap* m, const void* ptr, int D, int T, int Y, int X, int BH) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return DIT_ERR_CUDA;
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(X), static_cast<cuuint64_t>(Y),
+                        static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(X) * D * e,
+                           static_cast<cuuint64_t>(Y) * X * D * e, static_cast<cuuint64_t>(T) * Y * X * D * e};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / e), static_cast<cuuint32_t>(kNaBx),
+                       static_cast<cuuint32_t>(kNaBy), static_cast<cuuint32_t>(kNaBt), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
 // Number of SMs of the current device (cached per device).
 int sm_count(int* out) {
   static std::atomic<int> cache[64] = {};
@@ -105,14 +125,14 @@ int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
 // The forward kernel re-splits registers between warpgroups with setmaxnreg; the increase
 // only completes if the block was launched with at least the registers the split adds up to.
 // Refuse to launch a build where that does not hold (it would wait forever).
-template <int D, bool FP8>
+template <int D, bool FP8, bool NA>
 int check_register_split() {
   using C = AttnCfg<D, FP8>;
   static std::atomic<int> verdict{0};   // 0 unknown, 1 ok, 2 bad
   int v = verdict.load();
   if (v == 0) {
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8>) != cudaSuccess) return DIT_ERR_CUDA;
+    if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8, NA>) != cudaSuccess) return DIT_ERR_CUDA;
     const long long launched = static_cast<long long>(attr.numRegs) * C::kThreads;
     const long long wanted = 2LL * 128 * C::kRegsSoftmax + 128LL * C::kRegsCtl;
     v = (attr.numRegs == C::kRegsLaunch && launched >= wanted) ? 1 : 2;
@@ -121,29 +141,42 @@ int check_register_split() {
   return v == 1 ? DIT_OK : DIT_ERR_UNSUPPORTED;
 }
 
-template <int D, bool FP8>
+template <int D, bool FP8, bool NA = false>
 int launch_attn(const void* q, const void* k, const void* v, const AttnParams& prm, cudaStream_t st) {
   using C = AttnCfg<D, FP8>;
   static std::atomic<uint64_t> attr_done{0};
-  int rc = check_register_split<D, FP8>();
+  int rc = check_register_split<D, FP8, NA>();
   if (rc != DIT_OK) return rc;
-  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8>, C::kSmemBytes, attr_done);
+  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8, NA>, C::kSmemBytes, attr_done);
   if (rc != DIT_OK) return rc;
   CUtensorMap tq, tk, tv;
   const int BH = prm.B * prm.H;
-  if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH, prm.seg_q)) != DIT_OK) return rc;
-  if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
-  if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
   AttnParams pr = prm;
-  pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
-  pr.n_units = pr.n_qblk * prm.H * prm.B;
+  if constexpr (NA) {
+    if ((rc = make_map_na(&tq, q, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
+    if ((rc = make_map_na(&tk, k, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
+    if ((rc = make_map_na(&tv, v, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
+    pr.na_nbt = (prm.na_T + kNaBt - 1) / kNaBt;
+    pr.na_nby2 = (prm.na_Y + 2 * kNaBy - 1) / (2 * kNaBy);
+    pr.na_nbx = (prm.na_X + kNaBx - 1) / kNaBx;
+    const long long units = static_cast<long long>(BH) * pr.na_nbt * pr.na_nby2 * pr.na_nbx;
+    if (units > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+    pr.n_qblk = 0;
+    pr.n_units = static_cast<int>(units);
+  } else {
+    if ((rc = make_map(&tq, q, FP8, D, prm.S_q, BH, prm.seg_q)) != DIT_OK) return rc;
+    if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
+    if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
+    pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
+    pr.n_units = pr.n_qblk * prm.H * prm.B;
+  }
   int sms = 0;
   if ((rc = sm_count(&sms)) != DIT_OK) return rc;
   // persistent: at most one CTA per SM, minus the SMs reserved for concurrent kernels
   const int reserve = g_sm_reserve.load();
   const int slots = sms - reserve > 1 ? sms - reserve : 1;
   const int grid = pr.n_units < slots ? pr.n_units : slots;
-  attn_fwd_kernel<D, FP8><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, pr);
+  attn_fwd_kernel<D, FP8, NA><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, pr);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
@@ -262,6 +295,7 @@ int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, floa
   }
 
   AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
   prm.B = B; prm.H = H; prm.S_q = S_q; prm.S_kv = S_kv; prm.k0 = k0; prm.k1 = k1;
   prm.scale = scale;
   prm.descale = fp8 ? descale_qkv : nullptr;
@@ -319,6 +353,41 @@ int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, flo
   if (seg < 1) return DIT_ERR_INVALID_ARG;
   return attn_chunk_impl(q, k, v, out, lse, B, H, S, S, D, 0, S, scale, dtype, out_dtype, descale_qkv, stream,
                          false, BlockScales(), seg);
+}
+
+int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int T, int Y,
+                 int X, int D, int Kt, int Ky, int Kx, float scale, void* stream) {
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || T < 1 || Y < 1 || X < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
+  if (Kt < 1 || Ky < 1 || Kx < 1 || Kt % 2 == 0 || Ky % 2 == 0 || Kx % 2 == 0 || Kt > T || Ky > Y || Kx > X)
+    return DIT_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
+  const long long S = static_cast<long long>(T) * Y * X;
+  if (S > 0x7FFFFFFFLL || static_cast<long long>(B) * H * S > (1LL << 40)) return DIT_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16)) return DIT_ERR_MISALIGNED;
+  if (lse != nullptr && !aligned(lse, 4)) return DIT_ERR_MISALIGNED;
+  const size_t rows = static_cast<size_t>(B) * H * S, bytes = rows * D * 2;
+  if (overlaps(out, bytes, q, bytes) || overlaps(out, bytes, k, bytes) || overlaps(out, bytes, v, bytes))
+    return DIT_ERR_INVALID_ARG;
+  if (lse != nullptr && (overlaps(lse, rows * 4, out, bytes) || overlaps(lse, rows * 4, q, bytes) ||
+                         overlaps(lse, rows * 4, k, bytes) || overlaps(lse, rows * 4, v, bytes)))
+    return DIT_ERR_INVALID_ARG;
+  AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.B = B; prm.H = H; prm.S_q = static_cast<int>(S); prm.S_kv = static_cast<int>(S);
+  prm.k0 = 0; prm.k1 = static_cast<int>(S);
+  prm.scale = scale;
+  prm.out = out;
+  prm.lse = lse;
+  prm.seg_q = prm.S_q;
+  prm.seg_kv = prm.S_kv;
+  prm.na_T = T; prm.na_Y = Y; prm.na_X = X;
+  prm.na_Kt = Kt; prm.na_Ky = Ky; prm.na_Kx = Kx;
+  prm.timeout_ns = g_timeout_ns.load();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_attn<64, false, true>(q, k, v, prm, st);
+  return launch_attn<128, false, true>(q, k, v, prm, st);
 }
 
 int dit_swap01_chunks(const void* src, void* dst, long long d0, long long d1, long long chunk_bytes,
