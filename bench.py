@@ -239,6 +239,24 @@ class Step:
             f += self.w.flops
         return f
 
+    def run_heads(self, stream, g0: int, g1: int):
+        """The bf16 part of the step (full forward, chunks, merge) on the flattened heads
+        [g0, g1) of [B*H, S, D]: heads are independent, so a slice is a valid call with B = 1
+        and H = g1 - g0 on offset pointers."""
+        lsa, w = self.lsa, self.w
+        S, D, n = w.S, w.D, g1 - g0
+
+        def sl(t, per_row):
+            return t.data_ptr() + g0 * S * per_row * t.element_size()
+        q, k, v = sl(self.q, D), sl(self.k, D), sl(self.v, D)
+        lsa.dit_attn_fwd(q, k, v, sl(self.out, D), sl(self.lse, 1), 1, n, S, D, w.scale, lsa.DIT_BF16, None, stream)
+        for (a, b), (po, pl) in zip(self.bounds, self.parts):
+            lsa.dit_attn_fwd_chunk(q, k, v, sl(po, D), sl(pl, 1), 1, n, S, S, D, a, b, w.scale, lsa.DIT_BF16,
+                                   lsa.DIT_FP32, None, stream)
+        if self.bounds:
+            lsa.dit_attn_merge([sl(p[0], D) for p in self.parts], [sl(p[1], 1) for p in self.parts],
+                               sl(self.mout, D), sl(self.mlse, 1), 1, n, S, D, lsa.DIT_FP32, lsa.DIT_BF16, stream)
+
     def run(self, stream, ev=None):
         lsa, w = self.lsa, self.w
         B, H, S, D = w.B, w.H, w.S, w.D
@@ -257,6 +275,11 @@ class Step:
                                B, H, S, D, lsa.DIT_FP32, lsa.DIT_BF16, stream)
             if ev is not None:
                 ev[3].record(stream)
+        self.run_fp8(stream, ev)
+
+    def run_fp8(self, stream, ev=None):
+        lsa, w = self.lsa, self.w
+        B, H, S, D = w.B, w.H, w.S, w.D
         if self.fp8:
             n = B * H * S * D
             for i, x in enumerate((self.q, self.k, self.v)):
@@ -317,6 +340,7 @@ def run_ours(args, rank, local_rank, world):
     # the outputs, all inside the timed region
     e2e = run_e2e(args, lsa, step, data, stream, dev, ranks)
     ring = run_ring_fused(lsa, step, stream, ranks) if step.bounds else None
+    na = run_na3d_context(lsa, dev, stream, ranks)
 
     ranks.close()
     if rank != 0:
@@ -373,11 +397,62 @@ def run_ours(args, rank, local_rank, world):
     if ring is not None:
         ring["chunks_plus_merge_ms"] = round((statistics.mean(chunk_ms) + statistics.mean(merge_ms)), 4)
         line["ring_fused"] = ring
+    line["na3d"] = na
     line["clocks"] = clk.summary()
     line["e2e"] = e2e
     if world == 1 and not args.skip_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
     print(json.dumps(line), flush=True)
+
+
+def na3d_tiles(grid, kernel) -> int:
+    """KV tiles the neighborhood kernel visits over all units of one head (its own rule:
+    units of two 4x4x8 bricks stacked along y, windows rounded out to bricks)."""
+    def ws(i, K, L):
+        return min(max(i - K // 2, 0), L - K)
+
+    def span(a, ext, K, L, b):
+        last = min(a + ext, L) - 1
+        return (ws(last, K, L) + K + b - 1) // b - ws(a, K, L) // b
+    T, Y, X = grid
+    return sum(span(t, 4, kernel[0], T, 4) * span(y, 8, kernel[1], Y, 4) * span(x, 8, kernel[2], X, 8)
+               for t in range(0, T, 4) for y in range(0, Y, 8) for x in range(0, X, 8))
+
+
+def run_na3d_context(lsa, dev, stream, ranks, reps: int = 10):
+    """3-D neighborhood attention on the video token grid (21 x 30 x 52, 40 heads, D = 128,
+    7 x 7 x 7 window), reported beside the step: its own kernel time, useful FLOP/s (keys in
+    windows) and executed FLOP/s (visited tiles).  Inputs are drawn on the device: this is a
+    kernel timing; parity is covered by the tests."""
+    import torch
+    grid, kernel, H, D = (21, 30, 52), (7, 7, 7), 40, 128
+    S = grid[0] * grid[1] * grid[2]
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    q, k, v = (torch.randn((1, H, S, D), generator=g, device=dev, dtype=torch.float32).to(torch.bfloat16)
+               for _ in range(3))
+    out = torch.empty_like(q)
+    lse = torch.empty((1, H, S), dtype=torch.float32, device=dev)
+    call = lambda: lsa.dit_na3d_fwd(q, k, v, out, lse, 1, H, *grid, D, *kernel, D ** -0.5, stream)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        stream.synchronize()
+        ranks.barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            call()
+        t1.record(stream)
+    stream.synchronize()
+    ms = ranks.max(t0.elapsed_time(t1)) / reps
+    useful = 4.0 * H * S * kernel[0] * kernel[1] * kernel[2] * D
+    executed = 4.0 * H * na3d_tiles(grid, kernel) * 256 * 128 * D
+    del q, k, v, out, lse
+    return {"grid": list(grid), "window": list(kernel), "heads": H, "D": D, "ms": round(ms, 4),
+            "useful_tflops": round(useful * ranks.world / (ms * 1e-3) / 1e12, 2),
+            "executed_tflops": round(executed * ranks.world / (ms * 1e-3) / 1e12, 2),
+            "tile_efficiency": round(useful / executed, 4), "call": "dit_na3d_fwd"}
 
 
 def run_ring_fused(lsa, step, stream, ranks, reps: int = 10):
@@ -426,15 +501,53 @@ def run_e2e(args, lsa, step, data, stream, dev, ranks):
         host_o8 = torch.empty(step.out8.shape, dtype=torch.bfloat16).pin_memory()
         outs += [(host_o8, step.out8)]
     n_steps = max(3, min(args.steps, 10))
+    BH = w.B * w.H
+    G = max(1, min(args.e2e_groups, BH))
+    cuts = [BH * g // G for g in range(G + 1)]
+    c_in, c_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    fp8_outs = [(h, d) for h, d in outs if step.fp8 and d is step.out8]
+    head_outs = [(h, d) for h, d in outs if not (step.fp8 and d is step.out8)]
+
+    def rows(t, g0, g1):
+        return t.view(BH, -1)[g0:g1]
 
     def one():
-        for h, d in zip(host_in, (step.q, step.k, step.v)):
-            d.copy_(h, non_blocking=True)
-        step.run(stream)
-        for h, d in outs:
-            h.copy_(d, non_blocking=True)
+        # Head groups in a three-stream pipeline: the H2D copy of group g+1 and the D2H copy
+        # of group g-1 run on the copy engines while the kernels of group g run.
+        start = torch.cuda.Event()
+        start.record(stream)
+        c_in.wait_event(start)
+        c_out.wait_event(start)
+        for g in range(G):
+            g0, g1 = cuts[g], cuts[g + 1]
+            with torch.cuda.stream(c_in):
+                for h, d in zip(host_in, (step.q, step.k, step.v)):
+                    rows(d, g0, g1).copy_(rows(h, g0, g1), non_blocking=True)
+                arrived = torch.cuda.Event()
+                arrived.record(c_in)
+            stream.wait_event(arrived)
+            step.run_heads(stream, g0, g1)
+            done = torch.cuda.Event()
+            done.record(stream)
+            c_out.wait_event(done)
+            with torch.cuda.stream(c_out):
+                for h, d in head_outs:
+                    rows(h, g0, g1).copy_(rows(d, g0, g1), non_blocking=True)
+        if step.fp8:          # per-tensor scales need the whole tensors: after the last group
+            step.run_fp8(stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            c_out.wait_event(done)
+            with torch.cuda.stream(c_out):
+                for h, d in fp8_outs:
+                    h.copy_(d, non_blocking=True)
+        end = torch.cuda.Event()
+        end.record(c_out)
+        stream.wait_event(end)
 
     with torch.cuda.stream(stream):
+        step.run(stream)                       # whole-tensor calls, for the check below
+        ref = [d.clone() for _, d in outs]
         one()
         stream.synchronize()
         ranks.barrier()
@@ -445,10 +558,15 @@ def run_e2e(args, lsa, step, data, stream, dev, ranks):
         t1.record(stream)
     stream.synchronize()
     ms = ranks.max(t0.elapsed_time(t1)) / n_steps
+    # the head-group calls must give the whole-tensor calls' results bit for bit
+    same = all(torch.equal(h, r.cpu()) for (h, _), r in zip(outs, ref))
+    del ref
     bi = sum(h.numel() * h.element_size() for h in host_in)
     bo = sum(h.numel() * h.element_size() for h, _ in outs)
     return {"value": round(step.flops * ranks.world / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-            "ms_per_step": round(ms, 3), "steps": n_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+            "ms_per_step": round(ms, 3), "steps": n_steps, "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+            "head_groups": G, "pipeline": "H2D / kernels / D2H on three streams, per head group",
+            "matches_whole_tensor_calls": bool(same)}
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
@@ -532,6 +650,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=6.0, help="CPU work per --impl reference step")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-groups", type=int, default=4,
+                    help="head groups of the end-to-end pipeline (copies of one group overlap kernels of another)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

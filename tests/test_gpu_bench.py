@@ -28,6 +28,19 @@ def test_bench_json_line_contract():
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["achieved"] > 0
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-4          # frac is rounded to 4 places
     assert d["e2e"]["h2d_bytes_per_step"] == 3 * 2 * 256 * 64 * 2 and d["e2e"]["d2h_bytes_per_step"] > 0
+    assert d["e2e"]["head_groups"] == 2 and d["e2e"]["matches_whole_tensor_calls"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["gpu_launches"] == 5 * 4                        # fwd + 2 chunks + merge per step
     assert d["merge_roofline"]["bound"] == "hbm"
+
+
+def test_bench_video_e2e_pipeline_matches():
+    """Video workload (bf16 + e4m3 variant): the head-group pipeline of the end-to-end leg
+    reproduces the whole-tensor calls bit for bit."""
+    cmd = [sys.executable, "bench.py", "--workload", "video", "--steps", "3", "--warmup", "3",
+           "--skip-cpu-baseline", "--e2e-groups", "5"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")][0]
+    assert d["e2e"]["head_groups"] == 5 and d["e2e"]["matches_whole_tensor_calls"] is True
+    assert d["device_status"] == 0
