@@ -502,8 +502,16 @@ def run_e2e(args, lsa, step, data, stream, dev, ranks):
         outs += [(host_o8, step.out8)]
     n_steps = max(3, min(args.steps, 10))
     BH = w.B * w.H
-    G = max(1, min(args.e2e_groups, BH))
-    cuts = [BH * g // G for g in range(G + 1)]
+    if args.e2e_groups > 0:
+        G = max(1, min(args.e2e_groups, BH))
+    else:
+        # as many whole heads per group as one wave of work units (256 query rows of one
+        # head, one per SM) holds: small groups overlap copies best, a partial second wave
+        # would leave SMs idle
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        per_group = max(1, sms // ((w.S + 255) // 256))
+        G = (BH + per_group - 1) // per_group
+    cuts = [min(BH, g * ((BH + G - 1) // G)) for g in range(G + 1)]
     c_in, c_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
     fp8_outs = [(h, d) for h, d in outs if step.fp8 and d is step.out8]
     head_outs = [(h, d) for h, d in outs if not (step.fp8 and d is step.out8)]
@@ -516,19 +524,22 @@ def run_e2e(args, lsa, step, data, stream, dev, ranks):
         # of group g-1 run on the copy engines while the kernels of group g run.
         start = torch.cuda.Event()
         start.record(stream)
-        c_in.wait_event(start)
-        c_out.wait_event(start)
+        for st in (c_in, c_out):
+            st.wait_event(start)
         for g in range(G):
             g0, g1 = cuts[g], cuts[g + 1]
+            if g1 <= g0:
+                continue
+            cs = stream
             with torch.cuda.stream(c_in):
                 for h, d in zip(host_in, (step.q, step.k, step.v)):
                     rows(d, g0, g1).copy_(rows(h, g0, g1), non_blocking=True)
                 arrived = torch.cuda.Event()
                 arrived.record(c_in)
-            stream.wait_event(arrived)
-            step.run_heads(stream, g0, g1)
+            cs.wait_event(arrived)
+            step.run_heads(cs, g0, g1)
             done = torch.cuda.Event()
-            done.record(stream)
+            done.record(cs)
             c_out.wait_event(done)
             with torch.cuda.stream(c_out):
                 for h, d in head_outs:
@@ -650,8 +661,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=6.0, help="CPU work per --impl reference step")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-groups", type=int, default=4,
-                    help="head groups of the end-to-end pipeline (copies of one group overlap kernels of another)")
+    ap.add_argument("--e2e-groups", type=int, default=0,
+                    help="head groups of the end-to-end pipeline (copies of one group overlap kernels of another);"
+                         " 0 = about one wave of work units per group")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -28,7 +28,7 @@ def test_bench_json_line_contract():
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s" and r["achieved"] > 0
     assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-4          # frac is rounded to 4 places
     assert d["e2e"]["h2d_bytes_per_step"] == 3 * 2 * 256 * 64 * 2 and d["e2e"]["d2h_bytes_per_step"] > 0
-    assert d["e2e"]["head_groups"] == 2 and d["e2e"]["matches_whole_tensor_calls"] is True
+    assert d["e2e"]["head_groups"] == 1 and d["e2e"]["matches_whole_tensor_calls"] is True
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["gpu_launches"] == 5 * 4                        # fwd + 2 chunks + merge per step
     assert d["merge_roofline"]["bound"] == "hbm"
