@@ -341,6 +341,8 @@ def run_ours(args, rank, local_rank, world):
     e2e = run_e2e(args, lsa, step, data, stream, dev, ranks)
     ring = run_ring_fused(lsa, step, stream, ranks) if step.bounds else None
     na = run_na3d_context(lsa, dev, stream, ranks)
+    seg = run_seg_context(lsa, step, stream, ranks)
+    fp8b = run_fp8_blocks_context(lsa, step, stream, ranks)
 
     ranks.close()
     if rank != 0:
@@ -398,6 +400,9 @@ def run_ours(args, rank, local_rank, world):
         ring["chunks_plus_merge_ms"] = round((statistics.mean(chunk_ms) + statistics.mean(merge_ms)), 4)
         line["ring_fused"] = ring
     line["na3d"] = na
+    if seg is not None:
+        line["ulysses_seg"] = seg
+    line["fp8_blocks"] = fp8b
     line["clocks"] = clk.summary()
     line["e2e"] = e2e
     if world == 1 and not args.skip_cpu_baseline:
@@ -453,6 +458,79 @@ def run_na3d_context(lsa, dev, stream, ranks, reps: int = 10):
             "useful_tflops": round(useful * ranks.world / (ms * 1e-3) / 1e12, 2),
             "executed_tflops": round(executed * ranks.world / (ms * 1e-3) / 1e12, 2),
             "tile_efficiency": round(useful / executed, 4), "call": "dit_na3d_fwd"}
+
+
+def _time_calls(call, stream, ranks, reps: int = 10) -> float:
+    """ms per call: CUDA events on the launching stream after 3 warm-up calls, max over ranks."""
+    import torch
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            call()
+        stream.synchronize()
+        ranks.barrier()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(reps):
+            call()
+        t1.record(stream)
+    stream.synchronize()
+    return ranks.max(t0.elapsed_time(t1)) / reps
+
+
+def run_seg_context(lsa, step, stream, ranks):
+    """dit_attn_fwd_seg on the step's Q/K/V laid out as a 4-way sequence all-to-all delivers
+    them ([4, B*H, S/4, D]), beside dit_attn_fwd on the plain layout: the segmented
+    addressing of the Ulysses path should cost nothing."""
+    import torch
+    w = step.w
+    B, H, S, D = w.B, w.H, w.S, w.D
+    P = 4
+    if S % P or (S // P) % 128:
+        return None
+    seg = S // P
+    lay = lambda x: x.reshape(B * H, P, seg, D).transpose(0, 1).contiguous()
+    q, k, v = lay(step.q), lay(step.k), lay(step.v)
+    out = torch.empty_like(q)
+    lse = torch.empty((P, B * H, seg), dtype=torch.float32, device=q.device)
+    ms_seg = _time_calls(lambda: lsa.dit_attn_fwd_seg(q, k, v, out, lse, B, H, S, D, seg, w.scale, lsa.DIT_BF16,
+                                                      lsa.DIT_BF16, None, stream), stream, ranks)
+    ms_plain = _time_calls(lambda: lsa.dit_attn_fwd(step.q, step.k, step.v, step.out, step.lse, B, H, S, D, w.scale,
+                                                    lsa.DIT_BF16, None, stream), stream, ranks)
+    same = bool(torch.equal(out.transpose(0, 1).reshape(B, H, S, D), step.out))
+    del q, k, v, out, lse
+    return {"segments": P, "seg_rows": seg, "ms": round(ms_seg, 4), "plain_layout_ms": round(ms_plain, 4),
+            "tflops": round(w.flops * ranks.world / (ms_seg * 1e-3) / 1e12, 2),
+            "bit_identical_to_plain": same, "call": "dit_attn_fwd_seg"}
+
+
+def run_fp8_blocks_context(lsa, step, stream, ranks):
+    """Per-block E4M3 on the step's Q/K/V: dit_quant_fp8_blocks of the three tensors (HBM-bound)
+    and dit_attn_fwd_fp8_blocks (against 2x the measured bf16 peak, the nominal e4m3 ratio)."""
+    import torch
+    w = step.w
+    B, H, S, D = w.B, w.H, w.S, w.D
+    if D != 128:
+        return None
+    nb = (S + 127) // 128
+    codes = [torch.empty((B, H, S, D), dtype=torch.uint8, device=step.q.device) for _ in range(3)]
+    ds = [torch.empty((B, H, nb), dtype=torch.float32, device=step.q.device) for _ in range(3)]
+    out = torch.empty_like(step.out)
+    lse = torch.empty_like(step.lse)
+
+    def quant():
+        for x, c, d in zip((step.q, step.k, step.v), codes, ds):
+            lsa.dit_quant_fp8_blocks(x, c, d, B, H, S, D, stream)
+    ms_q = _time_calls(quant, stream, ranks)
+    ms_f = _time_calls(lambda: lsa.dit_attn_fwd_fp8_blocks(*codes, *ds, out, lse, B, H, S, S, D, 0, S, w.scale,
+                                                          lsa.DIT_BF16, stream), stream, ranks)
+    peaks, _ = load_peaks()
+    tf = w.flops * ranks.world / (ms_f * 1e-3) / 1e12
+    qbytes = 3 * B * H * S * D * 3 + 3 * B * H * nb * 4
+    del codes, ds, out, lse
+    return {"quant_ms_3_tensors": round(ms_q, 4), "quant_gbs": round(qbytes / (ms_q * 1e-3) / 1e9, 1),
+            "fwd_ms": round(ms_f, 4), "fwd_tflops": round(tf, 2),
+            "fwd_frac_of_2x_bf16_peak": round(tf / (2 * peaks["bf16_tflops"]), 4),
+            "calls": "3 x dit_quant_fp8_blocks, dit_attn_fwd_fp8_blocks"}
 
 
 def run_ring_fused(lsa, step, stream, ranks, reps: int = 10):
