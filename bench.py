@@ -353,7 +353,13 @@ def run_ours(args, rank, local_rank, world):
     value = total_flops / (elapsed_ms * 1e-3) / 1e12
     avg_full = statistics.mean(full_ms)
     achieved = w.flops / (avg_full * 1e-3) / 1e12
-    peak = peaks["bf16_tflops"]
+    # Denominator: the burst cuBLAS figure for a kernel timed alone, the sustained one (seconds
+    # of back-to-back GEMMs under the power cap) when the kernel runs inside a timed region of
+    # a second or more of continuous work, as here with the default step count.
+    long_region = elapsed_ms >= 1000.0 and "bf16_tflops_sustained" in peaks
+    peak = peaks["bf16_tflops_sustained"] if long_region else peaks["bf16_tflops"]
+    peak_src = (f"{peaks_src} bf16_tflops_sustained (kernel timed inside {elapsed_ms / 1000:.1f} s of "
+                f"back-to-back steps)" if long_region else f"{peaks_src} bf16_tflops (burst)")
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -376,7 +382,8 @@ def run_ours(args, rank, local_rank, world):
                    "parallelism": "replicas%d" % world},
         "roofline": {"bound": "tensor", "kernel": "attn_fwd_kernel<128,bf16> (dit_attn_fwd)",
                      "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "peak_source": f"{peaks_src} bf16_tflops (burst)",
+                     "frac": round(achieved / peak, 4), "peak_source": peak_src,
+                     "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
                      "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
                      "traffic": profiled_traffic(),
                      "algorithmic_bytes": 4 * w.B * w.H * w.S * w.D * 2 + w.B * w.H * w.S * 4},
