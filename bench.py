@@ -419,13 +419,14 @@ def run_ours(args, rank, local_rank, world):
 
 def na3d_tiles(grid, kernel) -> int:
     """KV tiles the neighborhood kernel visits over all units of one head (its own rule:
-    units of two 4x4x8 bricks stacked along y, windows rounded out to bricks)."""
+    units of two 4x4x8 bricks stacked along y; the union of their windows covered by bricks
+    laid from the union's origin)."""
     def ws(i, K, L):
         return min(max(i - K // 2, 0), L - K)
 
     def span(a, ext, K, L, b):
         last = min(a + ext, L) - 1
-        return (ws(last, K, L) + K + b - 1) // b - ws(a, K, L) // b
+        return (ws(last, K, L) + K - ws(a, K, L) + b - 1) // b
     T, Y, X = grid
     return sum(span(t, 4, kernel[0], T, 4) * span(y, 8, kernel[1], Y, 4) * span(x, 8, kernel[2], X, 8)
                for t in range(0, T, 4) for y in range(0, Y, 8) for x in range(0, X, 8))

@@ -87,9 +87,9 @@ struct AttnParams {
 // clamp(i - K/2, 0, L - K); the 3-D neighborhood is the product over (t, y, x).
 // A 128-row tile is a brick of kNaBt x kNaBy x kNaBx tokens, loaded by one 5-D TMA box
 // (x fastest), so tile row c is the token (c / 32, (c / 8) % 4, c % 8) of the brick.  A unit
-// is two bricks stacked along y; it visits every KV brick that the windows of its queries
-// touch (the union of windows, rounded out to bricks), and each row masks the keys outside
-// its own window.
+// is two bricks stacked along y; its KV tiles are bricks laid from the origin of the union of
+// its queries' windows (TMA boxes may start at any token; only the innermost D coordinate has
+// an alignment rule), and each row masks the keys outside its own window.
 // ---------------------------------------------------------------------------------------
 constexpr int kNaBt = 4, kNaBy = 4, kNaBx = 8;
 
@@ -98,24 +98,24 @@ __device__ __forceinline__ int na_wstart(int i, int K, int L) { return min(max(i
 struct NaUnit {
   int bh;
   int qt, qy, qx;        // token origin of Q brick 0 (brick 1 is kNaBy further along y)
-  int bt0, by0, bx0;     // first KV brick (in bricks)
+  int ut, uy, ux;        // token origin of the union of the unit's windows
   int nt, ny, nx;        // KV bricks along t, y, x
   __device__ __forceinline__ int n() const { return nt * ny * nx; }
   // token origin of KV tile j (x fastest, then y, then t)
   __device__ __forceinline__ void kv_origin(int j, int& t, int& y, int& x) const {
     const int jx = j % nx, jy = (j / nx) % ny, jt = j / (nx * ny);
-    t = (bt0 + jt) * kNaBt;
-    y = (by0 + jy) * kNaBy;
-    x = (bx0 + jx) * kNaBx;
+    t = ut + jt * kNaBt;
+    y = uy + jy * kNaBy;
+    x = ux + jx * kNaBx;
   }
 };
 
-// KV bricks covering the windows of the queries [a, min(a + ext, L)) along one dimension.
+// Union [first, first + len) of the windows of the queries [a, min(a + ext, L)) along one
+// dimension (window starts never decrease with the position), covered by `count` bricks of b.
 __device__ __forceinline__ void na_span(int a, int ext, int K, int L, int b, int& first, int& count) {
   const int last = min(a + ext, L) - 1;
-  const int lo = na_wstart(a, K, L), hi = na_wstart(last, K, L) + K;
-  first = lo / b;
-  count = (hi + b - 1) / b - first;
+  first = na_wstart(a, K, L);
+  count = (na_wstart(last, K, L) + K - first + b - 1) / b;
 }
 
 __device__ __forceinline__ NaUnit na_unit(const AttnParams& p, int u) {
@@ -127,9 +127,9 @@ __device__ __forceinline__ NaUnit na_unit(const AttnParams& p, int u) {
   w.qt = it * kNaBt;
   w.qy = iy * 2 * kNaBy;
   w.qx = ix * kNaBx;
-  na_span(w.qt, kNaBt, p.na_Kt, p.na_T, kNaBt, w.bt0, w.nt);
-  na_span(w.qy, 2 * kNaBy, p.na_Ky, p.na_Y, kNaBy, w.by0, w.ny);
-  na_span(w.qx, kNaBx, p.na_Kx, p.na_X, kNaBx, w.bx0, w.nx);
+  na_span(w.qt, kNaBt, p.na_Kt, p.na_T, kNaBt, w.ut, w.nt);
+  na_span(w.qy, 2 * kNaBy, p.na_Ky, p.na_Y, kNaBy, w.uy, w.ny);
+  na_span(w.qx, kNaBx, p.na_Kx, p.na_X, kNaBx, w.ux, w.nx);
   return w;
 }
 
