@@ -418,7 +418,8 @@ int dit_quant_fp8_blocks(const void* x_bf16, void* x_fp8, float* descales, int B
       overlaps(descales, static_cast<size_t>(grid) * 4, x_fp8, n))
     return DIT_ERR_INVALID_ARG;
   quant_e4m3_rows_kernel<<<static_cast<unsigned>(grid), kQuantRowThreads, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint16_t*>(x_bf16), S, D, static_cast<int>(nblk), static_cast<uint8_t*>(x_fp8), descales);
+      static_cast<const uint16_t*>(x_bf16), S, D, static_cast<int>(nblk), static_cast<uint8_t*>(x_fp8), descales,
+      g_timeout_ns.load());
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 

@@ -140,18 +140,23 @@ __global__ void __launch_bounds__(kQuantThreads) quant_e4m3_kernel(const uint16_
 }
 
 // Per-block scales: one CTA per block of 128 consecutive rows of one (b, h) of a [B,H,S,D]
-// tensor (the last block of a head may be shorter).  The block (at most 128 x 128 bf16 =
-// 32 KB) is read once into registers, its absolute maximum reduced, and the codes written:
-// one HBM read and one write per element.  An all-zero block gets descale 0 (it holds only
+// tensor (the last block of a head may be shorter).  The block is contiguous in memory (at
+// most 128 x 128 bf16 = 32 KB): one bulk copy brings it into shared memory, the CTA reduces
+// its absolute maximum there and writes the codes: one HBM read and one write per element,
+// with several CTAs' copies in flight per SM.  An all-zero block gets descale 0 (it holds only
 // zero codes; a consumer can tell it apart from a block whose maximum is 448) and codes of
 // x / 1, the per-tensor rule for an all-zero tensor.
 constexpr int kQuantBlockRows = 128;
-constexpr int kQuantRowThreads = 256;          // 8 16-byte vectors per thread at D = 128 (measured:
-                                               // faster than 512 threads x 4)
+constexpr int kQuantRowThreads = 256;
+constexpr int kQuantRowVecs = kQuantBlockRows * 128 / 8;     // 16-byte vectors of a full D = 128 block
 
 __global__ void __launch_bounds__(kQuantRowThreads) quant_e4m3_rows_kernel(const uint16_t* __restrict__ x, int S,
                                                                            int D, int nblk, uint8_t* __restrict__ x8,
-                                                                           float* __restrict__ descales) {
+                                                                           float* __restrict__ descales,
+                                                                           unsigned long long timeout_ns) {
+  __shared__ __align__(128) uint4 buf[kQuantRowVecs];
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
   __shared__ float red[kQuantRowThreads / 32];
   const long long bh = blockIdx.x / nblk;
   const int i = static_cast<int>(blockIdx.x - bh * nblk);
@@ -159,15 +164,26 @@ __global__ void __launch_bounds__(kQuantRowThreads) quant_e4m3_rows_kernel(const
   const int rows = min(kQuantBlockRows, S - r0);
   const long long base = (bh * S + r0) * static_cast<long long>(D);      // first element
   const int nvec = rows * D / 8;                                         // D % 8 == 0
-  constexpr int kPer = kQuantBlockRows * 128 / 8 / kQuantRowThreads;     // vectors per thread (D <= 128)
-  uint4 a[kPer];
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(nvec) * 16u);
+    bulk_load(buf, x + base, static_cast<uint32_t>(nvec) * 16u, &bar);
+  }
+  const bool ok = mbar_wait(&bar, 0, &abort_flag, timeout_ns, 0xB0);
+  if (!__syncthreads_and(ok)) {
+    // the copy this CTA issued must land before its shared memory goes away
+    if (threadIdx.x == 0) mbar_wait_drain(&bar, 0, timeout_ns);
+    return;
+  }
   float m = 0.0f;
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int idx = threadIdx.x + k * kQuantRowThreads;
-    a[k] = make_uint4(0u, 0u, 0u, 0u);
-    if (idx < nvec) a[k] = __ldg(reinterpret_cast<const uint4*>(x + base) + idx);
-    const uint32_t w[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+  for (int idx = threadIdx.x; idx < nvec; idx += kQuantRowThreads) {
+    const uint4 a = buf[idx];
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
       m = fmaxf(m, fabsf(bf16_bits_to_float(w[e] & 0xFFFFu)));
@@ -178,20 +194,17 @@ __global__ void __launch_bounds__(kQuantRowThreads) quant_e4m3_rows_kernel(const
   const float descale = (amax > 0.0f) ? __fdiv_rn(amax, 448.0f) : 1.0f;
   const float rcp = __frcp_rn(descale);
   if (threadIdx.x == 0) descales[blockIdx.x] = (amax > 0.0f) ? descale : 0.0f;
+  for (int idx = threadIdx.x; idx < nvec; idx += kQuantRowThreads) {
+    const uint4 a = buf[idx];
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+    uint32_t packed[2];
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int idx = threadIdx.x + k * kQuantRowThreads;
-    if (idx < nvec) {
-      const uint32_t w[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
-      uint32_t packed[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h)
-        packed[h] = pack_e4m3x4(quot_e4m3(bf16_bits_to_float(w[2 * h] & 0xFFFFu), descale, rcp),
-                                quot_e4m3(bf16_bits_to_float(w[2 * h] >> 16), descale, rcp),
-                                quot_e4m3(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), descale, rcp),
-                                quot_e4m3(bf16_bits_to_float(w[2 * h + 1] >> 16), descale, rcp));
-      reinterpret_cast<uint2*>(x8 + base)[idx] = make_uint2(packed[0], packed[1]);
-    }
+    for (int h = 0; h < 2; ++h)
+      packed[h] = pack_e4m3x4(quot_e4m3(bf16_bits_to_float(w[2 * h] & 0xFFFFu), descale, rcp),
+                              quot_e4m3(bf16_bits_to_float(w[2 * h] >> 16), descale, rcp),
+                              quot_e4m3(bf16_bits_to_float(w[2 * h + 1] & 0xFFFFu), descale, rcp),
+                              quot_e4m3(bf16_bits_to_float(w[2 * h + 1] >> 16), descale, rcp));
+    reinterpret_cast<uint2*>(x8 + base)[idx] = make_uint2(packed[0], packed[1]);
   }
 }
 
