@@ -1,15 +1,16 @@
-// Per-tensor absmax quantisation of bf16 to FP8-E4M3 (the input side of the FP8 attention
-// variant).
+// Absmax quantisation of bf16 to FP8-E4M3 (the input side of the FP8 attention variant).
 //
 // The AMD ROCm summary page (xDiT on Radeon AI PRO R9700S) names an FP8 attention backend
 // and notes that FP8 runs natively and changes outputs relative to BF16.  The pages fix no
-// scaling scheme; this library uses one scale per tensor:
+// scaling scheme; this library uses one scale per tensor (and, as a finer variant, one per
+// 128-row block of a head):
 //     amax = max |x|,  descale = amax / 448 (1 if amax = 0),  code = e4m3_rn_satfinite(x / descale)
-// with an IEEE fp32 division, so that the codes are reproducible bit for bit.
+// with the codes of an IEEE fp32 division, reproducible bit for bit (see quot_e4m3).
 //
-// Two launches, both HBM-bound: (1) per-block partial maxima into a small workspace,
-// (2) every block reduces the partials (a few KB, L2-resident), then quantises its share
-// with 16-byte loads and 8-byte stores.  Block 0 also writes descale.
+// Per tensor: two launches, both HBM-bound: (1) per-block partial maxima into a small
+// workspace, (2) every block reduces the partials (a few KB, L2-resident), then quantises its
+// share with 16-byte loads and 8-byte stores.  Block 0 also writes descale.
+// Per block: one launch, one CTA per block (quant_e4m3_rows_kernel below).
 #pragma once
 
 #include <cuda_bf16.h>
