@@ -144,6 +144,45 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int T, int Y, int X, int D, int Kt, int Ky, int Kx, float scale, void* stream);
 
 /*
+ * dit_attn_fwd_parts - the Ulysses step as one kernel over (peer) memory: the sequence is held
+ * in n_parts blocks of part_rows rows, block p by tensors [B, part_H, part_rows, D] (typically
+ * rank p's own Q, K, V, reachable through peer addresses over NVLink).  The call computes full
+ * attention over all n_parts * part_rows rows for heads [h0, h0 + H): Q/K/V tiles of those heads
+ * are loaded by TMA straight from each block's tensors, and every output row (and LSE) is
+ * written into the block it belongs to, out_parts[p][b, h0 + h, row, :] (lse_parts[p][b, h0 + h,
+ * row]).  Run with h0 = rank * H on every rank (H = part_H / P), it replaces the two all-to-all
+ * exchanges of the USP Ulysses dimension (xDiT overview page, section 3.2.2) and the re-layout
+ * copies around them.  Loads are plain TMA (no multicast); stores are plain global stores.
+ *
+ *   q_parts, k_parts, v_parts, out_parts  HOST arrays of n_parts device pointers (bf16,
+ *             16-byte aligned), read during the call only; lse_parts: host array of n_parts fp32
+ *             device pointers, or NULL.
+ *   1 <= n_parts <= 8; part_rows % 128 == 0 when n_parts > 1 (else DIT_ERR_UNSUPPORTED);
+ *   0 <= h0, h0 + H <= part_H; D = 64 or 128.
+ *   Ordering across GPUs is the caller's: every block's Q/K/V must be written before any
+ *   launch that reads it starts, and the outputs are complete when every launch that writes
+ *   them has finished (e.g. a barrier before and after).
+ */
+int dit_attn_fwd_parts(const void* const* q_parts, const void* const* k_parts,
+                       const void* const* v_parts, void* const* out_parts, float* const* lse_parts,
+                       int n_parts, int B, int part_H, int h0, int H, int part_rows, int D,
+                       float scale, void* stream);
+
+/*
+ * dit_ipc_export / dit_ipc_import / dit_ipc_close - share device buffers between the processes
+ * of one node (one per GPU), for dit_attn_fwd_parts on peer memory.
+ *   dit_ipc_export: the CUDA IPC handle (64 bytes, written to `handle`) of the allocation that
+ *     holds `ptr`, and ptr's byte offset inside it.
+ *   dit_ipc_import: opens a handle exported by another process (peer access enabled lazily)
+ *     and returns the mapped allocation (`base`) and base + offset (`ptr`).
+ *   dit_ipc_close: unmaps an imported allocation (`base` from dit_ipc_import).
+ * A handle cannot be imported by the process that exported it.  DIT_ERR_CUDA on failure.
+ */
+int dit_ipc_export(const void* ptr, void* handle, long long* offset);
+int dit_ipc_import(const void* handle, long long offset, void** ptr, void** base);
+int dit_ipc_close(void* base);
+
+/*
  * dit_swap01_chunks - dst[i1][i0] = src[i0][i1] for a [d0][d1] grid of chunks of chunk_bytes
  * bytes each (the batch/peer transpose around a Ulysses all-to-all when B > 1).
  *   src, dst  device buffers of d0 * d1 * chunk_bytes bytes, 16-byte aligned, not overlapping.

@@ -57,6 +57,10 @@ def _load() -> ctypes.CDLL:
     lib.dit_attn_fwd_seg.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp]
     lib.dit_swap01_chunks.argtypes = [vp, vp, ll, ll, ll, vp]
     lib.dit_na3d_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp]
+    lib.dit_attn_fwd_parts.argtypes = [ctypes.POINTER(vp)] * 5 + [i, i, i, i, i, i, i, f, vp]
+    lib.dit_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ll)]
+    lib.dit_ipc_import.argtypes = [vp, ll, ctypes.POINTER(vp), ctypes.POINTER(vp)]
+    lib.dit_ipc_close.argtypes = [vp]
     lib.dit_attn_fwd_fp8_blocks.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, i, vp]
     lib.dit_status_str.argtypes = [i]
     lib.dit_status_str.restype = ctypes.c_char_p
@@ -146,6 +150,38 @@ def dit_attn_fwd_seg(q, k, v, out, lse, B: int, H: int, S: int, D: int, seg: int
                      dtype: int = 0, out_dtype: int = 0, descale_qkv=None, stream=None) -> None:
     _check(lib.dit_attn_fwd_seg(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D, seg, float(scale),
                                 dtype, out_dtype, _ptr(descale_qkv), _stream(stream)), "dit_attn_fwd_seg")
+
+
+def dit_attn_fwd_parts(q_parts: Sequence, k_parts: Sequence, v_parts: Sequence, out_parts: Sequence,
+                       lse_parts: Optional[Sequence], B: int, part_H: int, h0: int, H: int, part_rows: int, D: int,
+                       scale: float, stream=None) -> None:
+    n = len(q_parts)
+    arr = lambda xs: (ctypes.c_void_p * n)(*[_ptr(x) for x in xs])
+    lse_arr = None if lse_parts is None else arr(lse_parts)
+    _check(lib.dit_attn_fwd_parts(arr(q_parts), arr(k_parts), arr(v_parts), arr(out_parts),
+                                  ctypes.cast(lse_arr, ctypes.POINTER(ctypes.c_void_p)) if lse_arr is not None else None,
+                                  n, B, part_H, h0, H, part_rows, D, float(scale), _stream(stream)),
+           "dit_attn_fwd_parts")
+
+
+def dit_ipc_export(ptr) -> Tuple[bytes, int]:
+    """(64-byte CUDA IPC handle of the allocation holding ptr, byte offset of ptr in it)."""
+    h = ctypes.create_string_buffer(64)
+    off = ctypes.c_longlong(0)
+    _check(lib.dit_ipc_export(_ptr(ptr), h, ctypes.byref(off)), "dit_ipc_export")
+    return h.raw, off.value
+
+
+def dit_ipc_import(handle: bytes, offset: int) -> Tuple[int, int]:
+    """(device address, mapped allocation base) of a buffer exported by another process."""
+    p, b = ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib.dit_ipc_import(ctypes.create_string_buffer(handle, 64), int(offset), ctypes.byref(p), ctypes.byref(b)),
+           "dit_ipc_import")
+    return p.value, b.value
+
+
+def dit_ipc_close(base: int) -> None:
+    _check(lib.dit_ipc_close(base), "dit_ipc_close")
 
 
 def dit_na3d_fwd(q, k, v, out, lse, B: int, H: int, T: int, Y: int, X: int, D: int, Kt: int, Ky: int, Kx: int,

@@ -13,6 +13,8 @@ benchmark) and quick timing: prints the average time per call from CUDA events. 
     quant_blocks  dit_quant_fp8_blocks of one tensor
     fp8           dit_attn_fwd on E4M3 codes (per-tensor descales)
     seg           dit_attn_fwd_seg with 4 segments
+    parts         dit_attn_fwd_parts: 4 ranks' blocks in separate buffers, one launch per rank
+                  (each for a quarter of the heads; on one GPU the launches run one after another)
     na3d          dit_na3d_fwd on a T x Y x X grid
 
 Inputs are N(0,1) drawn on the device (torch), rounded to bf16: this is a timing and
@@ -29,7 +31,8 @@ def main(argv=None) -> None:
     import long_sequence_attention_b200 as lsa
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["attn", "chunk", "merge", "quant", "quant_blocks", "fp8", "seg", "na3d"])
+    ap.add_argument("case", choices=["attn", "chunk", "merge", "quant", "quant_blocks", "fp8", "seg", "parts",
+                                     "na3d"])
     ap.add_argument("--reps", type=int, default=2)
     ap.add_argument("--shape", default="1,24,16896,128", help="B,H,S,D")
     ap.add_argument("--grid", default="21,30,52", help="T,Y,X (na3d; S = T*Y*X)")
@@ -87,6 +90,18 @@ def main(argv=None) -> None:
         out, lse = torch.empty_like(q), torch.empty((B, H, S), device=dev)
         call = lambda: lsa.dit_attn_fwd_seg(q, k, v, out, lse, B, H, S, D, seg, scale, lsa.DIT_BF16, lsa.DIT_BF16,
                                             None, st)
+    elif a.case == "parts":
+        P = 4
+        rows = S // P
+        blocks = [[torch.randn((B, H, rows, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(3)]
+                  for _ in range(P)]
+        outs = [torch.empty((B, H, rows, D), dtype=torch.bfloat16, device=dev) for _ in range(P)]
+        lses = [torch.empty((B, H, rows), device=dev) for _ in range(P)]
+
+        def call():
+            for r in range(P):
+                lsa.dit_attn_fwd_parts([b[0] for b in blocks], [b[1] for b in blocks], [b[2] for b in blocks], outs,
+                                       lses, B, H, r * (H // P), H // P, rows, D, scale, st)
     else:
         out, lse = torch.empty_like(q), torch.empty((B, H, S), device=dev)
         call = lambda: lsa.dit_na3d_fwd(q, k, v, out, lse, B, H, *grid, D, *window, scale, st)

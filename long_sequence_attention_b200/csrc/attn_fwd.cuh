@@ -77,7 +77,24 @@ struct AttnParams {
   int na_T, na_Y, na_X;
   int na_Kt, na_Ky, na_Kx;
   int na_nbt, na_nby2, na_nbx;
+  // Parts (the PARTS instantiation only): the sequence is n_parts blocks of part_rows rows,
+  // block p held by tensors [B, part_H, part_rows, D] at (possibly a peer GPU's) addresses;
+  // this launch computes heads [part_h0, part_h0 + H) over the whole sequence and writes the
+  // rows of block p into out_parts[p] / lse_parts[p] (same [B, part_H, part_rows] layout).
+  int n_parts, part_rows, part_H, part_h0;
+  void* out_parts[8];
+  float* lse_parts[8];
   unsigned long long timeout_ns;
+};
+
+constexpr int kMaxParts = 8;
+
+// Tensor maps of one launch: one each for Q, K, V, or one per part.
+template <int NM>
+struct MapSet {
+  CUtensorMap q[NM];
+  CUtensorMap k[NM];
+  CUtensorMap v[NM];
 };
 
 // ---------------------------------------------------------------------------------------
@@ -302,10 +319,12 @@ __device__ __forceinline__ void exp_pass(const uint32_t (&s)[128], float cl, flo
   sum = lo + hi;
 }
 
-template <int D, bool FP8, bool NA = false>
+template <int D, bool FP8, bool NA = false, bool PARTS = false>
 __global__ void __launch_bounds__(384, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                    const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+    attn_fwd_kernel(const __grid_constant__ MapSet<PARTS ? kMaxParts : 1> maps, const AttnParams p) {
+  const CUtensorMap& tm_q = maps.q[0];
+  const CUtensorMap& tm_k = maps.k[0];
+  const CUtensorMap& tm_v = maps.v[0];
   using C = AttnCfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -364,9 +383,17 @@ __global__ void __launch_bounds__(384, 1)
   if (warp == C::kTmaWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      if constexpr (PARTS) {
+        for (int pt = 0; pt < p.n_parts; ++pt) {
+          tma_prefetch_desc(&maps.q[pt]);
+          tma_prefetch_desc(&maps.k[pt]);
+          tma_prefetch_desc(&maps.v[pt]);
+        }
+      } else {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+      }
       int k_issued = 0, v_issued = 0, q_issued = 0;   // running counts over all units
       int g0 = 0;                                      // running KV tile count at unit start
       bool ok = true;
@@ -387,7 +414,13 @@ __global__ void __launch_bounds__(384, 1)
             if constexpr (NA)
               tma_load_5d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner, w.qx,
                           w.qy + t * kNaBy, w.qt, bh);
-            else
+            else if constexpr (PARTS) {
+              // row -> (part, row in part); rows past the last part read as zero (past its end)
+              const int row = q0 + t * C::kBM;
+              const int pt = min(row / p.part_rows, p.n_parts - 1);
+              tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &maps.q[pt], bar_q_full, b * C::kBoxInner,
+                          row - pt * p.part_rows, bh % p.H, bh / p.H);
+            } else
               tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner,
                           (q0 + t * C::kBM) % p.seg_q, bh, (q0 + t * C::kBM) / p.seg_q);
           }
@@ -406,7 +439,11 @@ __global__ void __launch_bounds__(384, 1)
             if constexpr (NA)
               tma_load_5d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks, b * C::kBoxInner,
                           ox, oy, ot, bh);
-            else
+            else if constexpr (PARTS) {
+              const int pt = min(kv_row / p.part_rows, p.n_parts - 1);
+              tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &maps.k[pt], bar_k_full + ks,
+                          b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
+            } else
               tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks,
                           b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
           }
@@ -420,7 +457,11 @@ __global__ void __launch_bounds__(384, 1)
             if constexpr (NA)
               tma_load_5d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs, b * C::kBoxInner,
                           ox, oy, ot, bh);
-            else
+            else if constexpr (PARTS) {
+              const int pt = min(kv_row / p.part_rows, p.n_parts - 1);
+              tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &maps.v[pt], bar_v_full + vs,
+                          b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
+            } else
               tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs,
                           b * C::kBoxInner, kv_row % p.seg_kv, bh, kv_row / p.seg_kv);
           }
@@ -708,9 +749,19 @@ __global__ void __launch_bounds__(384, 1)
       const int grow = q_start + t * C::kBM + row;
       bool store;
       size_t row_idx;
+      void* out_base = p.out;
+      float* lse_base = p.lse;
       if constexpr (NA) {
         store = qt < p.na_T && qy < p.na_Y && qx < p.na_X;
         row_idx = static_cast<size_t>(bh) * p.S_q + (static_cast<size_t>(qt) * p.na_Y + qy) * p.na_X + qx;
+      } else if constexpr (PARTS) {
+        // the row goes to the part that holds it, at its head in the part's full-head layout
+        store = grow < p.S_q;
+        const int pt = min(grow / p.part_rows, p.n_parts - 1);
+        out_base = p.out_parts[pt];
+        lse_base = p.lse_parts[pt];
+        row_idx = (static_cast<size_t>(bh / p.H) * p.part_H + p.part_h0 + bh % p.H) * p.part_rows +
+                  (grow - pt * p.part_rows);
       } else {
         store = grow < p.S_q;
         row_idx = (static_cast<size_t>(grow / p.seg_q) * p.B * p.H + bh) * p.seg_q + grow % p.seg_q;
@@ -722,7 +773,7 @@ __global__ void __launch_bounds__(384, 1)
       // this range's partial, w = exp(lse - M) / L with M the larger LSE and L the weight sum.
       float w_old = 0.0f, w_new = 1.0f, lse_out = lse_c;
       if (p.accumulate && store) {
-        const float la = p.lse[row_idx];
+        const float la = lse_base[row_idx];
         const float M = fmaxf(la, lse_c);
         const float ea = __expf(la - M);                     // 0 for an empty accumulator
         const float ec = __expf(lse_c - M);
@@ -740,7 +791,7 @@ __global__ void __launch_bounds__(384, 1)
           if (p.accumulate && w_old != 0.0f) {
             // (an empty accumulator, w_old = 0, is overwritten below without being read, so
             // whatever its buffer holds cannot leak in)
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_elem + cc * 32);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out_base) + row_elem + cc * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               const float4 a = dst[i];
@@ -750,7 +801,7 @@ __global__ void __launch_bounds__(384, 1)
                                    fmaf(a.w, w_old, __uint_as_float(o[4 * i + 3]) * inv_l));
             }
           } else if (p.out_fp32 || p.accumulate) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + row_elem + cc * 32);
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out_base) + row_elem + cc * 32);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
               dst[i] = make_float4(__uint_as_float(o[4 * i]) * inv_l, __uint_as_float(o[4 * i + 1]) * inv_l,
@@ -760,13 +811,13 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i)
               w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + row_elem + cc * 32);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out_base) + row_elem + cc * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
           }
         }
       }
-      if (store && p.lse != nullptr) p.lse[row_idx] = lse_out;
+      if (store && lse_base != nullptr) lse_base[row_idx] = lse_out;
       // The O reads above end with tcgen05.wait::ld; the next unit's first P.V (which
       // overwrites O_t) is issued only after this warpgroup publishes that unit's P_t.
     }

@@ -42,6 +42,23 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+typedef CUresult (*MemGetAddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+
+// cuMemGetAddressRange through the same entry-point lookup (the allocation holding a pointer,
+// needed to export a pointer that lies inside a larger allocation).
+MemGetAddressRangeFn addr_range_fn() {
+  static std::once_flag once;
+  static MemGetAddressRangeFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<MemGetAddressRangeFn>(p);
+  });
+  return fn;
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -125,14 +142,14 @@ int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
 // The forward kernel re-splits registers between warpgroups with setmaxnreg; the increase
 // only completes if the block was launched with at least the registers the split adds up to.
 // Refuse to launch a build where that does not hold (it would wait forever).
-template <int D, bool FP8, bool NA>
+template <int D, bool FP8, bool NA, bool PARTS>
 int check_register_split() {
   using C = AttnCfg<D, FP8>;
   static std::atomic<int> verdict{0};   // 0 unknown, 1 ok, 2 bad
   int v = verdict.load();
   if (v == 0) {
     cudaFuncAttributes attr;
-    if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8, NA>) != cudaSuccess) return DIT_ERR_CUDA;
+    if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8, NA, PARTS>) != cudaSuccess) return DIT_ERR_CUDA;
     const long long launched = static_cast<long long>(attr.numRegs) * C::kThreads;
     const long long wanted = 2LL * 128 * C::kRegsSoftmax + 128LL * C::kRegsCtl;
     v = (attr.numRegs == C::kRegsLaunch && launched >= wanted) ? 1 : 2;
@@ -141,18 +158,62 @@ int check_register_split() {
   return v == 1 ? DIT_OK : DIT_ERR_UNSUPPORTED;
 }
 
-template <int D, bool FP8, bool NA = false>
-int launch_attn(const void* q, const void* k, const void* v, const AttnParams& prm, cudaStream_t st) {
+// Parts launch: per part p a 4-D map (D, part_rows, H, B) over heads [h0, h0 + H) of the
+// part's [B, part_H, part_rows, D] tensor (the address may belong to a peer GPU).
+int make_map_part(CUtensorMap* m, const void* ptr, int D, int part_rows, int H, int B, int part_H, int h0) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return DIT_ERR_CUDA;
+  const cuuint64_t e = 2;
+  const char* base = static_cast<const char*>(ptr) + static_cast<size_t>(h0) * part_rows * D * e;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(part_rows), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(B)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(part_rows) * D * e,
+                           static_cast<cuuint64_t>(part_H) * part_rows * D * e};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / e), 128, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<char*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
+// Q/K/V pointers of a launch: one tensor each, or one per part.
+struct QKV {
+  const void* q[kMaxParts];
+  const void* k[kMaxParts];
+  const void* v[kMaxParts];
+};
+
+template <int D, bool FP8, bool NA = false, bool PARTS = false>
+int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
   using C = AttnCfg<D, FP8>;
   static std::atomic<uint64_t> attr_done{0};
-  int rc = check_register_split<D, FP8, NA>();
+  int rc = check_register_split<D, FP8, NA, PARTS>();
   if (rc != DIT_OK) return rc;
-  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8, NA>, C::kSmemBytes, attr_done);
+  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8, NA, PARTS>, C::kSmemBytes, attr_done);
   if (rc != DIT_OK) return rc;
-  CUtensorMap tq, tk, tv;
+  MapSet<PARTS ? kMaxParts : 1> maps;
+  std::memset(&maps, 0, sizeof(maps));
+  CUtensorMap& tq = maps.q[0];
+  CUtensorMap& tk = maps.k[0];
+  CUtensorMap& tv = maps.v[0];
+  const void* q = in.q[0];
+  const void* k = in.k[0];
+  const void* v = in.v[0];
   const int BH = prm.B * prm.H;
   AttnParams pr = prm;
-  if constexpr (NA) {
+  if constexpr (PARTS) {
+    for (int pt = 0; pt < prm.n_parts; ++pt) {
+      if ((rc = make_map_part(&maps.q[pt], in.q[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
+        return rc;
+      if ((rc = make_map_part(&maps.k[pt], in.k[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
+        return rc;
+      if ((rc = make_map_part(&maps.v[pt], in.v[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
+        return rc;
+    }
+    pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
+    pr.n_units = pr.n_qblk * prm.H * prm.B;
+  } else if constexpr (NA) {
     if ((rc = make_map_na(&tq, q, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
     if ((rc = make_map_na(&tk, k, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
     if ((rc = make_map_na(&tv, v, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
@@ -176,7 +237,7 @@ int launch_attn(const void* q, const void* k, const void* v, const AttnParams& p
   const int reserve = g_sm_reserve.load();
   const int slots = sms - reserve > 1 ? sms - reserve : 1;
   const int grid = pr.n_units < slots ? pr.n_units : slots;
-  attn_fwd_kernel<D, FP8, NA><<<grid, C::kThreads, C::kSmemBytes, st>>>(tq, tk, tv, pr);
+  attn_fwd_kernel<D, FP8, NA, PARTS><<<grid, C::kThreads, C::kSmemBytes, st>>>(maps, pr);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
@@ -311,9 +372,13 @@ int attn_chunk_impl(const void* q, const void* k, const void* v, void* out, floa
   prm.seg_q = seg > 0 ? seg : S_q;
   prm.seg_kv = seg > 0 ? seg : S_kv;
   prm.timeout_ns = g_timeout_ns.load();
-  if (fp8) return launch_attn<128, true>(q, k, v, prm, st);
-  if (D == 64) return launch_attn<64, false>(q, k, v, prm, st);
-  return launch_attn<128, false>(q, k, v, prm, st);
+  QKV in;
+  in.q[0] = q;
+  in.k[0] = k;
+  in.v[0] = v;
+  if (fp8) return launch_attn<128, true>(in, prm, st);
+  if (D == 64) return launch_attn<64, false>(in, prm, st);
+  return launch_attn<128, false>(in, prm, st);
 }
 
 }  // namespace
@@ -386,8 +451,93 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
   prm.na_Kt = Kt; prm.na_Ky = Ky; prm.na_Kx = Kx;
   prm.timeout_ns = g_timeout_ns.load();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (D == 64) return launch_attn<64, false, true>(q, k, v, prm, st);
-  return launch_attn<128, false, true>(q, k, v, prm, st);
+  QKV in;
+  in.q[0] = q;
+  in.k[0] = k;
+  in.v[0] = v;
+  if (D == 64) return launch_attn<64, false, true>(in, prm, st);
+  return launch_attn<128, false, true>(in, prm, st);
+}
+
+int dit_attn_fwd_parts(const void* const* q_parts, const void* const* k_parts, const void* const* v_parts,
+                       void* const* out_parts, float* const* lse_parts, int n_parts, int B, int part_H, int h0,
+                       int H, int part_rows, int D, float scale, void* stream) {
+  if (q_parts == nullptr || k_parts == nullptr || v_parts == nullptr || out_parts == nullptr)
+    return DIT_ERR_INVALID_ARG;
+  if (n_parts < 1 || n_parts > kMaxParts) return DIT_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || part_rows < 1 || h0 < 0 || h0 + H > part_H || B > 65535 || part_H > 65535)
+    return DIT_ERR_INVALID_ARG;
+  if (!(scale > 0.0f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
+  if (n_parts > 1 && part_rows % 128 != 0) return DIT_ERR_UNSUPPORTED;   // tiles must not straddle parts
+  const long long S = static_cast<long long>(n_parts) * part_rows;
+  if (S > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  const size_t part_bytes = static_cast<size_t>(B) * part_H * part_rows * D * 2;
+  for (int i = 0; i < n_parts; ++i) {
+    if (q_parts[i] == nullptr || k_parts[i] == nullptr || v_parts[i] == nullptr || out_parts[i] == nullptr)
+      return DIT_ERR_INVALID_ARG;
+    if (!aligned(q_parts[i], 16) || !aligned(k_parts[i], 16) || !aligned(v_parts[i], 16) ||
+        !aligned(out_parts[i], 16))
+      return DIT_ERR_MISALIGNED;
+    if (lse_parts != nullptr && (lse_parts[i] == nullptr || !aligned(lse_parts[i], 4))) return DIT_ERR_INVALID_ARG;
+    for (int j = 0; j < n_parts; ++j)
+      if (overlaps(out_parts[i], part_bytes, q_parts[j], part_bytes) ||
+          overlaps(out_parts[i], part_bytes, k_parts[j], part_bytes) ||
+          overlaps(out_parts[i], part_bytes, v_parts[j], part_bytes) ||
+          (i != j && overlaps(out_parts[i], part_bytes, out_parts[j], part_bytes)))
+        return DIT_ERR_INVALID_ARG;
+  }
+  AttnParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.B = B; prm.H = H; prm.S_q = static_cast<int>(S); prm.S_kv = static_cast<int>(S);
+  prm.k0 = 0; prm.k1 = static_cast<int>(S);
+  prm.scale = scale;
+  prm.n_parts = n_parts; prm.part_rows = part_rows; prm.part_H = part_H; prm.part_h0 = h0;
+  QKV in;
+  std::memset(&in, 0, sizeof(in));
+  for (int i = 0; i < n_parts; ++i) {
+    in.q[i] = q_parts[i];
+    in.k[i] = k_parts[i];
+    in.v[i] = v_parts[i];
+    prm.out_parts[i] = out_parts[i];
+    prm.lse_parts[i] = lse_parts != nullptr ? lse_parts[i] : nullptr;
+  }
+  prm.seg_q = prm.S_q;
+  prm.seg_kv = prm.S_kv;
+  prm.timeout_ns = g_timeout_ns.load();
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (D == 64) return launch_attn<64, false, false, true>(in, prm, st);
+  return launch_attn<128, false, false, true>(in, prm, st);
+}
+
+int dit_ipc_export(const void* ptr, void* handle, long long* offset) {
+  if (ptr == nullptr || handle == nullptr || offset == nullptr) return DIT_ERR_INVALID_ARG;
+  MemGetAddressRangeFn range = addr_range_fn();
+  if (range == nullptr) return DIT_ERR_CUDA;
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return DIT_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return DIT_ERR_CUDA;
+  std::memcpy(handle, &h, sizeof(h));
+  *offset = static_cast<long long>(reinterpret_cast<uintptr_t>(ptr) - static_cast<uintptr_t>(base));
+  return DIT_OK;
+}
+
+int dit_ipc_import(const void* handle, long long offset, void** ptr, void** base) {
+  if (handle == nullptr || ptr == nullptr || base == nullptr || offset < 0) return DIT_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  std::memcpy(&h, handle, sizeof(h));
+  void* b = nullptr;
+  if (cudaIpcOpenMemHandle(&b, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return DIT_ERR_CUDA;
+  *base = b;
+  *ptr = static_cast<char*>(b) + offset;
+  return DIT_OK;
+}
+
+int dit_ipc_close(void* base) {
+  if (base == nullptr) return DIT_ERR_INVALID_ARG;
+  return cudaIpcCloseMemHandle(base) == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
 int dit_swap01_chunks(const void* src, void* dst, long long d0, long long d1, long long chunk_bytes,

@@ -17,6 +17,11 @@ piece, [P, H/P, S/P, D] = [H, S/P, D].  With B > 1 the piece for one peer is str
 Requirements: H divisible by P; every rank holds the same S/P rows, a multiple of 128 (the
 kernel's tiles must not straddle two segments) unless P = 1; bf16 inputs.
 
+``ulysses_attention_peers`` does the same step with no all-to-all at all: one launch per rank
+reads its head group of every rank's Q/K/V straight from the peers' memory (TMA, no
+multicast) and stores each output row into the rank it belongs to (dit_attn_fwd_parts), the
+buffers shared through CUDA IPC handles.
+
 This module is plumbing: buffers and collectives.  The attention and the copies run in the
 library's kernels (or, in the CPU tests of this schedule, in the functions those tests pass
 in).
@@ -109,4 +114,91 @@ def ulysses_attention_dist(q, k, v, scale: Optional[float] = None, *, group=None
 
     out = back(out_seg, D).view(B, H, S_loc, D)
     lse = back(lse_seg, 1).view(B, H, S_loc) if with_lse else None
+    return out, lse
+
+
+class CudaPeerOps:
+    """Buffer sharing and the fused launch for ulysses_attention_peers, on the library."""
+
+    def __init__(self):
+        self._opened = {}                 # (rank, handle) -> (base of the mapped allocation)
+
+    def export(self, t):
+        from . import dit_ipc_export
+        return dit_ipc_export(t)
+
+    def import_(self, rank: int, handle: bytes, offset: int) -> int:
+        from . import dit_ipc_import
+        key = (rank, handle)
+        if key not in self._opened:
+            _, base = dit_ipc_import(handle, 0)
+            self._opened[key] = base
+        return self._opened[key] + offset
+
+    def close(self):
+        from . import dit_ipc_close
+        for base in self._opened.values():
+            dit_ipc_close(base)
+        self._opened.clear()
+
+    def sync(self):
+        import torch
+        torch.cuda.synchronize()
+
+    def launch(self, qs, ks, vs, outs, lses, B, H, h0, Hp, rows, D, scale):
+        from . import dit_attn_fwd_parts
+        dit_attn_fwd_parts(qs, ks, vs, outs, lses, B, H, h0, Hp, rows, D, scale)
+
+
+def ulysses_attention_peers(q, k, v, scale: Optional[float] = None, *, group=None, ops=None, out=None, lse=None):
+    """The Ulysses step as one kernel over peer memory (dit_attn_fwd_parts): no all-to-all.
+
+    q, k, v    [B,H,S_loc,D] bf16, this rank's rows of every head (ranks hold consecutive rows).
+    out, lse   optional output buffers [B,H,S_loc,D] bf16 / [B,H,S_loc] fp32 (allocated if None).
+    Every rank exports its q, k, v, out and lse through CUDA IPC, opens the others' (kept
+    open by `ops` across calls: pass the same CudaPeerOps to reuse them), and after a barrier
+    runs one launch for its head group [rank*H/P, (rank+1)*H/P): its tiles are loaded by TMA
+    from the ranks that hold the rows, and its output rows are stored into the ranks they
+    belong to.  A second barrier makes every rank's out complete before it returns.
+    Returns (out, lse) for this rank's rows.  Collective over `group`.
+    """
+    import torch
+    import torch.distributed as dist
+
+    B, H, S_loc, D = (int(x) for x in q.shape)
+    if tuple(k.shape) != (B, H, S_loc, D) or k.shape != v.shape:
+        raise ValueError("q, k and v must all be [B,H,S_loc,D]")
+    P = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    if H % P != 0:
+        raise ValueError(f"H = {H} heads do not divide over {P} ranks")
+    if P > 1 and S_loc % 128 != 0:
+        raise ValueError(f"S_loc = {S_loc} rows per rank must be a multiple of 128")
+    if P > 8:
+        raise ValueError("at most 8 ranks")
+    scale = (1.0 / D ** 0.5) if scale is None else float(scale)
+    ops = CudaPeerOps() if ops is None else ops
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S_loc), dtype=torch.float32, device=q.device)
+    mine = [q, k, v, out, lse]
+    exported = [ops.export(t) for t in mine]
+    everyone = [None] * P
+    dist.all_gather_object(everyone, (S_loc, exported), group=group)
+    if any(e[0] != S_loc for e in everyone):
+        raise ValueError("every rank must hold the same number of rows")
+    ptrs = []                                     # ptrs[p] = (q, k, v, out, lse) addresses of rank p
+    for p_, (_, handles) in enumerate(everyone):
+        if p_ == r:
+            ptrs.append([t.data_ptr() for t in mine])
+        else:
+            ptrs.append([ops.import_(p_, h, off) for h, off in handles])
+    Hp = H // P
+    ops.sync()
+    dist.barrier(group=group)                     # every rank's q, k, v are written
+    ops.launch([x[0] for x in ptrs], [x[1] for x in ptrs], [x[2] for x in ptrs], [x[3] for x in ptrs],
+               [x[4] for x in ptrs], B, H, r * Hp, Hp, S_loc, D, scale)
+    ops.sync()
+    dist.barrier(group=group)                     # every rank's rows of out are written
     return out, lse
