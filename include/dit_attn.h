@@ -144,29 +144,33 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int T, int Y, int X, int D, int Kt, int Ky, int Kx, float scale, void* stream);
 
 /*
- * dit_attn_fwd_parts - the Ulysses step as one kernel over (peer) memory: the sequence is held
- * in n_parts blocks of part_rows rows, block p by tensors [B, part_H, part_rows, D] (typically
- * rank p's own Q, K, V, reachable through peer addresses over NVLink).  The call computes full
- * attention over all n_parts * part_rows rows for heads [h0, h0 + H): Q/K/V tiles of those heads
- * are loaded by TMA straight from each block's tensors, and every output row (and LSE) is
- * written into the block it belongs to, out_parts[p][b, h0 + h, row, :] (lse_parts[p][b, h0 + h,
- * row]).  Run with h0 = rank * H on every rank (H = part_H / P), it replaces the two all-to-all
- * exchanges of the USP Ulysses dimension (xDiT overview page, section 3.2.2) and the re-layout
- * copies around them.  Loads are plain TMA (no multicast); stores are plain global stores.
+ * dit_attn_fwd_parts - attention whose inputs lie in blocks held by several ranks (possibly on
+ * other GPUs, through peer addresses over NVLink), one kernel, no exchange.  The keys are
+ * n_kv_parts blocks and the queries n_q_parts blocks of part_rows rows each; block p is held
+ * by tensors [B, part_H, part_rows, D].  The call computes, for heads [h0, h0 + H), full
+ * attention of all n_q_parts * part_rows query rows over all n_kv_parts * part_rows keys:
+ * Q/K/V tiles are loaded by TMA straight from the block that holds them, and every output row
+ * (and LSE) is written into the query block it belongs to, out_parts[p][b, h0 + h, row, :].
+ * Loads are plain TMA (no multicast); stores are plain global stores.
+ *  - Ulysses step of USP (xDiT overview page, section 3.2.2): n_q_parts = n_kv_parts = P, one
+ *    launch per rank with h0 = rank * H (H = part_H / P): replaces both all-to-alls and the
+ *    re-layout copies around them.
+ *  - Ring step of USP without the ring: n_q_parts = 1 (this rank's rows), n_kv_parts = P,
+ *    h0 = 0, H = part_H: every rank reads the other ranks' K/V in place.
  *
- *   q_parts, k_parts, v_parts, out_parts  HOST arrays of n_parts device pointers (bf16,
- *             16-byte aligned), read during the call only; lse_parts: host array of n_parts fp32
- *             device pointers, or NULL.
- *   1 <= n_parts <= 8; part_rows % 128 == 0 when n_parts > 1 (else DIT_ERR_UNSUPPORTED);
- *   0 <= h0, h0 + H <= part_H; D = 64 or 128.
- *   Ordering across GPUs is the caller's: every block's Q/K/V must be written before any
- *   launch that reads it starts, and the outputs are complete when every launch that writes
- *   them has finished (e.g. a barrier before and after).
+ *   q_parts, out_parts  HOST arrays of n_q_parts device pointers; k_parts, v_parts: HOST arrays
+ *             of n_kv_parts device pointers (bf16, 16-byte aligned); lse_parts: host array of
+ *             n_q_parts fp32 device pointers, or NULL.  The arrays are read during the call only.
+ *   1 <= n_q_parts, n_kv_parts <= 8; part_rows % 128 == 0 unless both are 1 (else
+ *   DIT_ERR_UNSUPPORTED); 0 <= h0, h0 + H <= part_H; D = 64 or 128.
+ *   Ordering across GPUs is the caller's: every block must be written before any launch that
+ *   reads it starts, and the outputs are complete when every launch that writes them has
+ *   finished (e.g. a barrier before and after).
  */
-int dit_attn_fwd_parts(const void* const* q_parts, const void* const* k_parts,
-                       const void* const* v_parts, void* const* out_parts, float* const* lse_parts,
-                       int n_parts, int B, int part_H, int h0, int H, int part_rows, int D,
-                       float scale, void* stream);
+int dit_attn_fwd_parts(const void* const* q_parts, int n_q_parts, const void* const* k_parts,
+                       const void* const* v_parts, int n_kv_parts, void* const* out_parts,
+                       float* const* lse_parts, int B, int part_H, int h0, int H, int part_rows,
+                       int D, float scale, void* stream);
 
 /*
  * dit_ipc_export / dit_ipc_import / dit_ipc_close - share device buffers between the processes

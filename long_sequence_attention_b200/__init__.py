@@ -57,7 +57,8 @@ def _load() -> ctypes.CDLL:
     lib.dit_attn_fwd_seg.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp]
     lib.dit_swap01_chunks.argtypes = [vp, vp, ll, ll, ll, vp]
     lib.dit_na3d_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp]
-    lib.dit_attn_fwd_parts.argtypes = [ctypes.POINTER(vp)] * 5 + [i, i, i, i, i, i, i, f, vp]
+    lib.dit_attn_fwd_parts.argtypes = [ctypes.POINTER(vp), i, ctypes.POINTER(vp), ctypes.POINTER(vp), i,
+                                       ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, f, vp]
     lib.dit_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ll)]
     lib.dit_ipc_import.argtypes = [vp, ll, ctypes.POINTER(vp), ctypes.POINTER(vp)]
     lib.dit_ipc_close.argtypes = [vp]
@@ -155,13 +156,14 @@ def dit_attn_fwd_seg(q, k, v, out, lse, B: int, H: int, S: int, D: int, seg: int
 def dit_attn_fwd_parts(q_parts: Sequence, k_parts: Sequence, v_parts: Sequence, out_parts: Sequence,
                        lse_parts: Optional[Sequence], B: int, part_H: int, h0: int, H: int, part_rows: int, D: int,
                        scale: float, stream=None) -> None:
-    n = len(q_parts)
-    arr = lambda xs: (ctypes.c_void_p * n)(*[_ptr(x) for x in xs])
-    lse_arr = None if lse_parts is None else arr(lse_parts)
-    _check(lib.dit_attn_fwd_parts(arr(q_parts), arr(k_parts), arr(v_parts), arr(out_parts),
-                                  ctypes.cast(lse_arr, ctypes.POINTER(ctypes.c_void_p)) if lse_arr is not None else None,
-                                  n, B, part_H, h0, H, part_rows, D, float(scale), _stream(stream)),
-           "dit_attn_fwd_parts")
+    """Query blocks q_parts (outputs out_parts, lse_parts) and key blocks k_parts / v_parts;
+    the counts are the lengths of the lists."""
+    def arr(xs):
+        return (ctypes.c_void_p * len(xs))(*[_ptr(x) for x in xs])
+    lse_arr = None if lse_parts is None else ctypes.cast(arr(lse_parts), ctypes.POINTER(ctypes.c_void_p))
+    _check(lib.dit_attn_fwd_parts(arr(q_parts), len(q_parts), arr(k_parts), arr(v_parts), len(k_parts),
+                                  arr(out_parts), lse_arr, B, part_H, h0, H, part_rows, D, float(scale),
+                                  _stream(stream)), "dit_attn_fwd_parts")
 
 
 def dit_ipc_export(ptr) -> Tuple[bytes, int]:

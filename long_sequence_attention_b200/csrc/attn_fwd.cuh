@@ -77,11 +77,11 @@ struct AttnParams {
   int na_T, na_Y, na_X;
   int na_Kt, na_Ky, na_Kx;
   int na_nbt, na_nby2, na_nbx;
-  // Parts (the PARTS instantiation only): the sequence is n_parts blocks of part_rows rows,
-  // block p held by tensors [B, part_H, part_rows, D] at (possibly a peer GPU's) addresses;
-  // this launch computes heads [part_h0, part_h0 + H) over the whole sequence and writes the
-  // rows of block p into out_parts[p] / lse_parts[p] (same [B, part_H, part_rows] layout).
-  int n_parts, part_rows, part_H, part_h0;
+  // Parts (the PARTS instantiation only): the keys are n_kv_parts blocks and the queries
+  // n_q_parts blocks of part_rows rows each, block p held by tensors [B, part_H, part_rows, D]
+  // at (possibly a peer GPU's) addresses; this launch computes heads [part_h0, part_h0 + H)
+  // and writes the rows of query block p into out_parts[p] / lse_parts[p] (same layout).
+  int n_q_parts, n_kv_parts, part_rows, part_H, part_h0;
   void* out_parts[8];
   float* lse_parts[8];
   unsigned long long timeout_ns;
@@ -384,8 +384,8 @@ __global__ void __launch_bounds__(384, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       if constexpr (PARTS) {
-        for (int pt = 0; pt < p.n_parts; ++pt) {
-          tma_prefetch_desc(&maps.q[pt]);
+        for (int pt = 0; pt < p.n_q_parts; ++pt) tma_prefetch_desc(&maps.q[pt]);
+        for (int pt = 0; pt < p.n_kv_parts; ++pt) {
           tma_prefetch_desc(&maps.k[pt]);
           tma_prefetch_desc(&maps.v[pt]);
         }
@@ -417,7 +417,7 @@ __global__ void __launch_bounds__(384, 1)
             else if constexpr (PARTS) {
               // row -> (part, row in part); rows past the last part read as zero (past its end)
               const int row = q0 + t * C::kBM;
-              const int pt = min(row / p.part_rows, p.n_parts - 1);
+              const int pt = min(row / p.part_rows, p.n_q_parts - 1);
               tma_load_4d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &maps.q[pt], bar_q_full, b * C::kBoxInner,
                           row - pt * p.part_rows, bh % p.H, bh / p.H);
             } else
@@ -440,7 +440,7 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_5d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks, b * C::kBoxInner,
                           ox, oy, ot, bh);
             else if constexpr (PARTS) {
-              const int pt = min(kv_row / p.part_rows, p.n_parts - 1);
+              const int pt = min(kv_row / p.part_rows, p.n_kv_parts - 1);
               tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &maps.k[pt], bar_k_full + ks,
                           b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
             } else
@@ -458,7 +458,7 @@ __global__ void __launch_bounds__(384, 1)
               tma_load_5d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs, b * C::kBoxInner,
                           ox, oy, ot, bh);
             else if constexpr (PARTS) {
-              const int pt = min(kv_row / p.part_rows, p.n_parts - 1);
+              const int pt = min(kv_row / p.part_rows, p.n_kv_parts - 1);
               tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &maps.v[pt], bar_v_full + vs,
                           b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
             } else
@@ -757,7 +757,7 @@ __global__ void __launch_bounds__(384, 1)
       } else if constexpr (PARTS) {
         // the row goes to the part that holds it, at its head in the part's full-head layout
         store = grow < p.S_q;
-        const int pt = min(grow / p.part_rows, p.n_parts - 1);
+        const int pt = min(grow / p.part_rows, p.n_q_parts - 1);
         out_base = p.out_parts[pt];
         lse_base = p.lse_parts[pt];
         row_idx = (static_cast<size_t>(bh / p.H) * p.part_H + p.part_h0 + bh % p.H) * p.part_rows +

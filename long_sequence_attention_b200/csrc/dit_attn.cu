@@ -203,9 +203,10 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
   const int BH = prm.B * prm.H;
   AttnParams pr = prm;
   if constexpr (PARTS) {
-    for (int pt = 0; pt < prm.n_parts; ++pt) {
+    for (int pt = 0; pt < prm.n_q_parts; ++pt)
       if ((rc = make_map_part(&maps.q[pt], in.q[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
         return rc;
+    for (int pt = 0; pt < prm.n_kv_parts; ++pt) {
       if ((rc = make_map_part(&maps.k[pt], in.k[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
         return rc;
       if ((rc = make_map_part(&maps.v[pt], in.v[pt], D, prm.part_rows, prm.H, prm.B, prm.part_H, prm.part_h0)) != DIT_OK)
@@ -459,46 +460,53 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
   return launch_attn<128, false, true>(in, prm, st);
 }
 
-int dit_attn_fwd_parts(const void* const* q_parts, const void* const* k_parts, const void* const* v_parts,
-                       void* const* out_parts, float* const* lse_parts, int n_parts, int B, int part_H, int h0,
-                       int H, int part_rows, int D, float scale, void* stream) {
+int dit_attn_fwd_parts(const void* const* q_parts, int n_q_parts, const void* const* k_parts,
+                       const void* const* v_parts, int n_kv_parts, void* const* out_parts, float* const* lse_parts,
+                       int B, int part_H, int h0, int H, int part_rows, int D, float scale, void* stream) {
   if (q_parts == nullptr || k_parts == nullptr || v_parts == nullptr || out_parts == nullptr)
     return DIT_ERR_INVALID_ARG;
-  if (n_parts < 1 || n_parts > kMaxParts) return DIT_ERR_INVALID_ARG;
+  if (n_q_parts < 1 || n_q_parts > kMaxParts || n_kv_parts < 1 || n_kv_parts > kMaxParts) return DIT_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || part_rows < 1 || h0 < 0 || h0 + H > part_H || B > 65535 || part_H > 65535)
     return DIT_ERR_INVALID_ARG;
   if (!(scale > 0.0f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
-  if (n_parts > 1 && part_rows % 128 != 0) return DIT_ERR_UNSUPPORTED;   // tiles must not straddle parts
-  const long long S = static_cast<long long>(n_parts) * part_rows;
-  if (S > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  if ((n_q_parts > 1 || n_kv_parts > 1) && part_rows % 128 != 0) return DIT_ERR_UNSUPPORTED;   // no straddling
+  const long long S_q = static_cast<long long>(n_q_parts) * part_rows;
+  const long long S_kv = static_cast<long long>(n_kv_parts) * part_rows;
+  if (S_q > 0x7FFFFFFFLL || S_kv > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
   const size_t part_bytes = static_cast<size_t>(B) * part_H * part_rows * D * 2;
-  for (int i = 0; i < n_parts; ++i) {
-    if (q_parts[i] == nullptr || k_parts[i] == nullptr || v_parts[i] == nullptr || out_parts[i] == nullptr)
-      return DIT_ERR_INVALID_ARG;
-    if (!aligned(q_parts[i], 16) || !aligned(k_parts[i], 16) || !aligned(v_parts[i], 16) ||
-        !aligned(out_parts[i], 16))
-      return DIT_ERR_MISALIGNED;
+  for (int i = 0; i < n_kv_parts; ++i) {
+    if (k_parts[i] == nullptr || v_parts[i] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned(k_parts[i], 16) || !aligned(v_parts[i], 16)) return DIT_ERR_MISALIGNED;
+  }
+  for (int i = 0; i < n_q_parts; ++i) {
+    if (q_parts[i] == nullptr || out_parts[i] == nullptr) return DIT_ERR_INVALID_ARG;
+    if (!aligned(q_parts[i], 16) || !aligned(out_parts[i], 16)) return DIT_ERR_MISALIGNED;
     if (lse_parts != nullptr && (lse_parts[i] == nullptr || !aligned(lse_parts[i], 4))) return DIT_ERR_INVALID_ARG;
-    for (int j = 0; j < n_parts; ++j)
+    for (int j = 0; j < n_q_parts; ++j)
       if (overlaps(out_parts[i], part_bytes, q_parts[j], part_bytes) ||
-          overlaps(out_parts[i], part_bytes, k_parts[j], part_bytes) ||
-          overlaps(out_parts[i], part_bytes, v_parts[j], part_bytes) ||
           (i != j && overlaps(out_parts[i], part_bytes, out_parts[j], part_bytes)))
+        return DIT_ERR_INVALID_ARG;
+    for (int j = 0; j < n_kv_parts; ++j)
+      if (overlaps(out_parts[i], part_bytes, k_parts[j], part_bytes) ||
+          overlaps(out_parts[i], part_bytes, v_parts[j], part_bytes))
         return DIT_ERR_INVALID_ARG;
   }
   AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
-  prm.B = B; prm.H = H; prm.S_q = static_cast<int>(S); prm.S_kv = static_cast<int>(S);
-  prm.k0 = 0; prm.k1 = static_cast<int>(S);
+  prm.B = B; prm.H = H; prm.S_q = static_cast<int>(S_q); prm.S_kv = static_cast<int>(S_kv);
+  prm.k0 = 0; prm.k1 = static_cast<int>(S_kv);
   prm.scale = scale;
-  prm.n_parts = n_parts; prm.part_rows = part_rows; prm.part_H = part_H; prm.part_h0 = h0;
+  prm.n_q_parts = n_q_parts; prm.n_kv_parts = n_kv_parts;
+  prm.part_rows = part_rows; prm.part_H = part_H; prm.part_h0 = h0;
   QKV in;
   std::memset(&in, 0, sizeof(in));
-  for (int i = 0; i < n_parts; ++i) {
-    in.q[i] = q_parts[i];
+  for (int i = 0; i < n_kv_parts; ++i) {
     in.k[i] = k_parts[i];
     in.v[i] = v_parts[i];
+  }
+  for (int i = 0; i < n_q_parts; ++i) {
+    in.q[i] = q_parts[i];
     prm.out_parts[i] = out_parts[i];
     prm.lse_parts[i] = lse_parts != nullptr ? lse_parts[i] : nullptr;
   }

@@ -16,6 +16,10 @@ so the ring asks the library to leave ``sm_reserve`` SMs free for NCCL's kernels
 Block lengths may differ between ranks (an S that does not divide by P): lengths are
 exchanged once on the host and every receive is posted with the sender's exact size.
 
+``ring_attention_peers`` computes the same result without moving blocks at all: one launch
+per rank reads every rank's K/V in place over peer memory (dit_attn_fwd_parts), the buffers
+shared through CUDA IPC handles.
+
 This module is plumbing around the C entry points: buffers, streams and the send/recv
 schedule.  All arithmetic runs in the library's kernels (or, in the CPU tests of this
 schedule, in the step functions those tests pass in).
@@ -154,3 +158,53 @@ def ring_attention_dist(q, k, v, scale: Optional[float] = None, *, group=None, d
             from . import dit_set_sm_reserve
             dit_set_sm_reserve(0)
     return ops.finish(acc, lse)
+
+
+def ring_attention_peers(q, k, v, scale: Optional[float] = None, *, group=None, ops=None, out=None, lse=None):
+    """The Ring dimension without a ring: one launch per rank reads every rank's K/V block in
+    place over peer memory (dit_attn_fwd_parts with this rank's queries as the only query
+    block), so no block travels and no partials are merged.
+
+    q, k, v    [B,H,S_loc,D] bf16: this rank's rows (ranks hold consecutive rows, equal S_loc,
+               a multiple of 128 when there is more than one rank).
+    Buffers are shared with CUDA IPC through `ops` (ulysses.CudaPeerOps; pass the same one
+    across calls to keep the peers' mappings open).  Barrier, launch, barrier.
+    Returns (out [B,H,S_loc,D] bf16, lse [B,H,S_loc] fp32).  Collective over `group`.
+    """
+    import torch
+    import torch.distributed as dist
+    from .ulysses import CudaPeerOps
+
+    B, H, S_loc, D = (int(x) for x in q.shape)
+    if tuple(k.shape) != (B, H, S_loc, D) or k.shape != v.shape:
+        raise ValueError("q, k and v must all be [B,H,S_loc,D]")
+    P = dist.get_world_size(group)
+    r = dist.get_rank(group)
+    if P > 8:
+        raise ValueError("at most 8 ranks")
+    if P > 1 and S_loc % 128 != 0:
+        raise ValueError(f"S_loc = {S_loc} rows per rank must be a multiple of 128")
+    scale = (1.0 / D ** 0.5) if scale is None else float(scale)
+    ops = CudaPeerOps() if ops is None else ops
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, S_loc), dtype=torch.float32, device=q.device)
+    everyone = [None] * P
+    dist.all_gather_object(everyone, (S_loc, [ops.export(k), ops.export(v)]), group=group)
+    if any(e[0] != S_loc for e in everyone):
+        raise ValueError("every rank must hold the same number of rows")
+    ks, vs = [], []
+    for p_, (_, handles) in enumerate(everyone):
+        if p_ == r:
+            ks.append(k.data_ptr())
+            vs.append(v.data_ptr())
+        else:
+            ks.append(ops.import_(p_, *handles[0]))
+            vs.append(ops.import_(p_, *handles[1]))
+    ops.sync()
+    dist.barrier(group=group)                     # every rank's k, v are written
+    ops.launch([q.data_ptr()], ks, vs, [out.data_ptr()], [lse.data_ptr()], B, H, 0, H, S_loc, D, scale)
+    ops.sync()
+    dist.barrier(group=group)                     # no rank overwrites its k, v while others read them
+    return out, lse

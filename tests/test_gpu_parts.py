@@ -105,3 +105,26 @@ def test_ipc_export_reports_offset_inside_allocation(cuda_lib):
     h0, off0 = cuda_lib.dit_ipc_export(big)
     h1, off1 = cuda_lib.dit_ipc_export(big[4096:])
     assert len(h0) == 64 and h0 == h1 and off1 - off0 == 4096
+
+
+@pytest.mark.parametrize("P,B,H,S_loc,D", [(2, 1, 3, 256, 128), (4, 2, 2, 128, 64), (1, 1, 2, 300, 128)])
+def test_ring_without_ring_equals_full_attention(cuda_lib, P, B, H, S_loc, D):
+    """Each virtual rank: its own rows as the only query block, every rank's K/V as key blocks."""
+    import torch
+    host, dev = _ranks(P, B, H, S_loc, D, seed=P + 50)
+    scale = 1.0 / np.sqrt(D)
+    outs, lses = [], []
+    for r in range(P):
+        o = torch.empty((B, H, S_loc, D), dtype=torch.bfloat16, device="cuda")
+        l = torch.empty((B, H, S_loc), dtype=torch.float32, device="cuda")
+        cuda_lib.dit_attn_fwd_parts([dev[r][0]], [d[1] for d in dev], [d[2] for d in dev], [o], [l],
+                                    B, H, 0, H, S_loc, D, scale)
+        outs.append(o)
+        lses.append(l)
+    torch.cuda.synchronize()
+    assert cuda_lib.dit_device_status() == 0
+    ro, rl = oracle.attention(*host, scale)
+    for r in range(P):
+        rows = slice(r * S_loc, (r + 1) * S_loc)
+        m = metrics(host_f64(outs[r]), ro[:, :, rows], lses[r].cpu().numpy().astype(np.float64), rl[:, :, rows])
+        assert_bf16_parity(m, (P, r))

@@ -122,3 +122,47 @@ def test_ring_single_rank_is_one_step(tmp_path):
     ref_o, ref_l = oracle.attention(q, k, v, 0.3)
     assert np.allclose(np.load(tmp_path / "out0.npy"), ref_o, rtol=0, atol=1e-6)
     assert json.load(open(tmp_path / "owners0.json")) == [0]
+
+
+def _ring_peers_worker(rank, world, port, buffers, out_dir):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import datetime
+    import torch.distributed as dist
+    from long_sequence_attention_b200.ring import ring_attention_peers
+    from test_ulysses_host import SharedMemoryPeerOps
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    ops = SharedMemoryPeerOps(rank, buffers, 0.3)
+    q, k, v, out, lse = buffers[rank]
+    ring_attention_peers(q, k, v, 0.3, ops=ops, out=out, lse=lse)
+    dist.destroy_process_group()
+    with open(os.path.join(out_dir, f"launch{rank}.txt"), "w") as f:
+        f.write(repr(ops.launches))
+
+
+@pytest.mark.parametrize("world,S_loc", [(2, 128), (3, 256)])
+def test_ring_peers_matches_oracle(tmp_path, world, S_loc):
+    """The ring without a ring: each rank's launch reads every rank's K/V block in place (here
+    shared CPU memory stands in for peer memory) and writes only its own rows."""
+    import torch
+    import torch.multiprocessing as mp
+    import oracle
+    B, H, D = 1, 2, 8
+    q, k, v, offs = _blocks([S_loc] * world, B=B, H=H, D=D)
+    buffers = []
+    for r in range(world):
+        rows = slice(offs[r], offs[r + 1])
+        bufs = [torch.from_numpy(np.ascontiguousarray(x[:, :, rows]).astype(np.float32)).share_memory_()
+                for x in (q, k, v)]
+        bufs.append(torch.full((B, H, S_loc, D), float("nan")).share_memory_())
+        bufs.append(torch.full((B, H, S_loc), float("nan")).share_memory_())
+        buffers.append(bufs)
+    mp.spawn(_ring_peers_worker, args=(world, _free_port(), buffers, str(tmp_path)), nprocs=world, join=True)
+    f32 = lambda x: x.astype(np.float32).astype(np.float64)
+    ro, rl = oracle.attention(f32(q), f32(k), f32(v), 0.3)
+    for r in range(world):
+        rows = slice(offs[r], offs[r + 1])
+        assert np.allclose(buffers[r][3].numpy(), ro[:, :, rows], rtol=0, atol=1e-6)
+        assert np.allclose(buffers[r][4].numpy(), rl[:, :, rows], rtol=0, atol=1e-5)
+        assert open(tmp_path / f"launch{r}.txt").read() == repr([(0, H)])
