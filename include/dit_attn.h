@@ -151,7 +151,7 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
  * attention of all n_q_parts * part_rows query rows over all n_kv_parts * part_rows keys:
  * Q/K/V tiles are loaded by TMA straight from the block that holds them, and every output row
  * (and LSE) is written into the query block it belongs to, out_parts[p][b, h0 + h, row, :].
- * Loads are plain TMA (no multicast); stores are plain global stores.
+ * Loads are plain TMA loads into the loading CTA's shared memory; stores are plain global stores.
  *  - Ulysses step of USP (xDiT overview page, section 3.2.2): n_q_parts = n_kv_parts = P, one
  *    launch per rank with h0 = rank * H (H = part_H / P): replaces both all-to-alls and the
  *    re-layout copies around them.

@@ -1,7 +1,7 @@
 // Device primitives for sm_100a, hand-written inline PTX.
 //
-// mbarrier (init, arrive, expect-tx, time-bounded wait), TMA tile loads (no multicast
-// anywhere in this library), tcgen05 tensor-core MMAs with TMEM accumulators, TMEM
+// mbarrier (init, arrive, expect-tx, time-bounded wait), TMA tile loads (each into the
+// issuing CTA's own shared memory only), tcgen05 tensor-core MMAs with TMEM accumulators, TMEM
 // allocation and TMEM <-> register copies, and the UMMA shared-memory / instruction
 // descriptors.  Descriptor bit layouts follow the PTX ISA description of tcgen05 matrix
 // descriptors (the same fields CUTLASS's cute/arch/mma_sm100_desc.hpp names).
@@ -104,7 +104,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 }
 
 // ------------------------------------------------------------------------------------
-// TMA (cp.async.bulk.tensor), tile mode, no multicast
+// TMA (cp.async.bulk.tensor), tile mode, destination: this CTA's shared memory
 // ------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -119,7 +119,7 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* map, uin
       : "memory");
 }
 
-// Untiled bulk copy global -> shared memory of this CTA (no multicast), completion on an
+// Untiled bulk copy global -> shared memory of this CTA only, completion on an
 // mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(

@@ -18,8 +18,8 @@ Requirements: H divisible by P; every rank holds the same S/P rows, a multiple o
 kernel's tiles must not straddle two segments) unless P = 1; bf16 inputs.
 
 ``ulysses_attention_peers`` does the same step with no all-to-all at all: one launch per rank
-reads its head group of every rank's Q/K/V straight from the peers' memory (TMA, no
-multicast) and stores each output row into the rank it belongs to (dit_attn_fwd_parts), the
+reads its head group of every rank's Q/K/V straight from the peers' memory (plain TMA
+loads into the reading CTA) and stores each output row into the rank it belongs to (dit_attn_fwd_parts), the
 buffers shared through CUDA IPC handles.
 
 This module is plumbing: buffers and collectives.  The attention and the copies run in the
