@@ -292,8 +292,28 @@ class Step:
                 ev[5].record(stream)
 
 
+def ensure_library():
+    """Build the in-tree CUDA library if it is missing or older than its sources (a no-op
+    otherwise), without importing the package first."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_lsa_build", os.path.join(ROOT, "long_sequence_attention_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
 def run_ours(args, rank, local_rank, world):
     import torch
+    if rank == 0 or world == 1:
+        ensure_library()
+    if world > 1:
+        # other ranks wait for rank 0's build through the file system: the library appears
+        # (os.replace) only when complete
+        deadline = time.time() + 900
+        lib = os.path.join(ROOT, "long_sequence_attention_b200", "libdit_attn.so")
+        while not os.path.exists(lib) and time.time() < deadline:
+            time.sleep(1.0)
     import long_sequence_attention_b200 as lsa
 
     dev = torch.device(f"cuda:{local_rank}")

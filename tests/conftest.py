@@ -14,9 +14,12 @@ def pytest_configure(config):
 
 @pytest.fixture(scope="session")
 def cuda_lib():
-    """The CUDA path's binding; GPU tests fail loudly if the library is missing."""
+    """The CUDA path's binding, built in-tree first if it is missing or older than its sources
+    (a no-op otherwise); GPU tests fail loudly if it cannot be built or loaded."""
     import torch
     if not torch.cuda.is_available():
         pytest.fail("GPU test selected but no CUDA device is visible")
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import long_sequence_attention_b200 as lsa
     return lsa

@@ -12,7 +12,7 @@ pytestmark = pytest.mark.gpu
 
 
 @pytest.mark.parametrize("case", ["attn", "chunk", "merge", "quant", "quant_blocks", "fp8", "seg", "parts", "na3d"])
-def test_case_runs(case):
+def test_case_runs(cuda_lib, case):
     cmd = [sys.executable, "-m", "long_sequence_attention_b200.cases", case, "--reps", "2",
            "--shape", "1,4,1024,128", "--grid", "2,8,16", "--window", "1,5,7"]
     out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
