@@ -173,24 +173,12 @@ __device__ __forceinline__ void apply_mask128(uint32_t (&s)[128], const uint32_t
     if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xFF800000u;
 }
 
-// exp2 on the FMA pipe for x <= 2^7: x = n + f with n = rint(x), f in [-1/2, 1/2];
-// 2^f by a degree-3 polynomial (minimax in relative error, max 7.5e-5; coefficients from
-// fit_exp2_poly.py); 2^n by adding n to the exponent field.  x is clamped at -125 so the
-// exponent never underflows (2^-125 stands in for 0; it only ever multiplies V values).
-__device__ __forceinline__ float exp2_fma(float x) {
-  x = fmaxf(x, -125.0f);
-  const float magic = 12582912.0f;  // 1.5 * 2^23: adding it rounds x to an integer
-  const float t = x + magic;
-  const float n = t - magic;
-  const float f = x - n;
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  // low bits of t hold n (two's complement); shifting them into the exponent field adds n
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
-// The same evaluation for two values at once with packed fp32x2 instructions.
+// exp2 on the FMA pipe for x <= 2^7, two values at once with packed fp32x2 instructions:
+// x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (minimax in
+// relative error, max 7.5e-5; coefficients from fit_exp2_poly.py); 2^n by adding n to the
+// exponent field.  x is clamped at -125 so the exponent never underflows (2^-125 stands in
+// for 0; it only ever multiplies V values).  Adding 1.5 * 2^23 rounds x to an integer whose
+// low bits (two's complement) are n; shifting them into the exponent field adds n.
 __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
   const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
   const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
