@@ -213,7 +213,9 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
         return rc;
     }
     pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
-    pr.n_units = pr.n_qblk * prm.H * prm.B;
+    const long long units = static_cast<long long>(pr.n_qblk) * prm.H * prm.B;
+    if (units > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+    pr.n_units = static_cast<int>(units);
   } else if constexpr (NA) {
     if ((rc = make_map_na(&tq, q, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
     if ((rc = make_map_na(&tk, k, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
@@ -230,7 +232,9 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
     if ((rc = make_map(&tk, k, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
     if ((rc = make_map(&tv, v, FP8, D, prm.S_kv, BH, prm.seg_kv)) != DIT_OK) return rc;
     pr.n_qblk = (prm.S_q + 2 * C::kBM - 1) / (2 * C::kBM);
-    pr.n_units = pr.n_qblk * prm.H * prm.B;
+    const long long units = static_cast<long long>(pr.n_qblk) * prm.H * prm.B;
+    if (units > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+    pr.n_units = static_cast<int>(units);
   }
   int sms = 0;
   if ((rc = sm_count(&sms)) != DIT_OK) return rc;
