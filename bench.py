@@ -362,6 +362,7 @@ def run_ours(args, rank, local_rank, world):
     ring = run_ring_fused(lsa, step, stream, ranks) if step.bounds else None
     na = run_na3d_context(lsa, dev, stream, ranks)
     seg = run_seg_context(lsa, step, stream, ranks)
+    parts = run_parts_context(lsa, step, stream, ranks)
     fp8b = run_fp8_blocks_context(lsa, step, stream, ranks)
 
     ranks.close()
@@ -429,6 +430,8 @@ def run_ours(args, rank, local_rank, world):
     line["na3d"] = na
     if seg is not None:
         line["ulysses_seg"] = seg
+    if parts is not None:
+        line["ulysses_peers_virtual"] = parts
     line["fp8_blocks"] = fp8b
     line["clocks"] = clk.summary()
     line["e2e"] = e2e
@@ -529,6 +532,33 @@ def run_seg_context(lsa, step, stream, ranks):
     return {"segments": P, "seg_rows": seg, "ms": round(ms_seg, 4), "plain_layout_ms": round(ms_plain, 4),
             "tflops": round(w.flops * ranks.world / (ms_seg * 1e-3) / 1e12, 2),
             "bit_identical_to_plain": same, "call": "dit_attn_fwd_seg"}
+
+
+def run_parts_context(lsa, step, stream, ranks):
+    """dit_attn_fwd_parts as 4 ranks would run it (each rank's rows in its own buffers, one
+    launch per rank for a quarter of the heads), here as 4 launches one after another on this
+    GPU: the fused Ulysses step's kernel time with all blocks local."""
+    import torch
+    w = step.w
+    B, H, S, D = w.B, w.H, w.S, w.D
+    P = 4
+    if S % P or (S // P) % 128 or H % P:
+        return None
+    rows = S // P
+    blocks = [[x[:, :, r * rows:(r + 1) * rows].contiguous() for x in (step.q, step.k, step.v)] for r in range(P)]
+    outs = [torch.empty((B, H, rows, D), dtype=torch.bfloat16, device=step.q.device) for _ in range(P)]
+    lses = [torch.empty((B, H, rows), dtype=torch.float32, device=step.q.device) for _ in range(P)]
+
+    def call():
+        for r in range(P):
+            lsa.dit_attn_fwd_parts([b[0] for b in blocks], [b[1] for b in blocks], [b[2] for b in blocks], outs, lses,
+                                   B, H, r * (H // P), H // P, rows, D, w.scale, stream)
+    ms = _time_calls(call, stream, ranks)
+    full = torch.cat(outs, dim=2)
+    same = bool(torch.equal(full, step.out))
+    del blocks, outs, lses, full
+    return {"ranks": P, "ms_all_launches": round(ms, 4), "tflops": round(w.flops * ranks.world / (ms * 1e-3) / 1e12, 2),
+            "bit_identical_to_plain": same, "call": "4 x dit_attn_fwd_parts (virtual ranks, blocks local)"}
 
 
 def run_fp8_blocks_context(lsa, step, stream, ranks):

@@ -11,7 +11,7 @@ Overlap: the send/recv of step t is posted before the attention of step t is enq
 the transfer of the next block runs beside the attention of the current one (over NVLink /
 NVSwitch with NCCL).  The attention kernel is persistent and fills every SM it runs on,
 so the ring asks the library to leave ``sm_reserve`` SMs free for NCCL's kernels
-(``dit_set_sm_reserve``) while it runs.
+(``dit_set_sm_reserve``) while it runs, and sets the reserve back to 0 when it returns.
 
 Block lengths may differ between ranks (an S that does not divide by P): lengths are
 exchanged once on the host and every receive is posted with the sender's exact size.
