@@ -14,8 +14,16 @@
 // exponentials of one tile overlap the tensor-core work of the other.  The kernel is
 // persistent: a grid of at most one CTA per SM walks the units u = blockIdx.x + k*gridDim.x
 // (query block fastest, so the CTAs running at the same time share a head's K/V in L2).
-// Barrier phases and ring stages follow a per-CTA running tile count g = it * n_kv + j, so
-// the next unit's Q load, its first S MMAs and this unit's epilogue overlap.
+// Barrier phases and ring stages follow a per-CTA running count g of KV tiles (every role
+// adds each unit's tile count, which varies per unit only in the neighborhood form), so the
+// next unit's Q load, its first S MMAs and this unit's epilogue overlap.
+//
+// Instantiations (template <D, FP8, NA, PARTS>): the dense form (bf16 D = 64 / 128, e4m3
+// D = 128, per-tensor or per-block scales, plain or sequence-segmented layouts, optional
+// running (O, LSE) accumulator); NA, 3-D neighborhood attention, where a tile is a 4x4x8
+// token brick and a unit visits only the KV bricks of its queries' windows, with per-row
+// window masks; PARTS, where the query and key rows lie in blocks held by several ranks
+// (possibly other GPUs) and every tile is loaded from the block that holds it.
 //
 // Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
