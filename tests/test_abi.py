@@ -133,3 +133,69 @@ def test_sm_reserve_validation(lib):
     assert lib.lib.dit_set_sm_reserve(1025) == 1
     assert lib.lib.dit_set_sm_reserve(8) == 0
     assert lib.lib.dit_set_sm_reserve(0) == 0
+
+
+# Every call below also carries at least one invalid argument (see the note above).
+def test_block_fp8_validation(lib):
+    qb = lib.lib.dit_quant_fp8_blocks
+    assert qb(None, Bp, L, 1, 2, 256, 128, None) == 1
+    assert qb(A, Bp, L, 1, 2, 256, 4, None) == 1                             # D < 8
+    assert qb(A, Bp, L, 1, 2, 256, 12, None) == 2                            # D % 8
+    assert qb(A, Bp, L, 1, 2, 256, 136, None) == 2                           # D > 128
+    assert qb(A + 2, Bp, L, 1, 2, 256, 128, None) == 3
+    assert qb(A, A + 64, L, 1, 2, 256, 128, None) == 1                       # codes overlap input
+    fb = lib.lib.dit_attn_fwd_fp8_blocks
+    assert fb(A, Bp, Cp, L, None, L + 4096, O, None, 1, 2, 256, 256, 128, 0, 256, 0.1, 0, None) == 1
+    assert fb(A, Bp, Cp, L, L + 1024, L + 4096, O, None, 1, 2, 256, 256, 128, 64, 256, 0.1, 0, None) == 2
+    assert fb(A, Bp, Cp, L, L + 1024, L + 4096, O, None, 1, 2, 256, 256, 64, 0, 256, 0.1, 0, None) == 2
+
+
+def test_seg_and_swap_validation(lib):
+    sg = lib.lib.dit_attn_fwd_seg
+    assert sg(A, Bp, Cp, O, L, 1, 2, 512, 128, 0, 0.1, 0, 0, None, None) == 1        # seg < 1
+    assert sg(A, Bp, Cp, O, L, 1, 2, 512, 128, 300, 0.1, 0, 0, None, None) == 1      # S % seg
+    assert sg(A, Bp, Cp, O, L, 1, 2, 512, 128, 64, 0.1, 0, 0, None, None) == 2       # seg % 128
+    sw = lib.lib.dit_swap01_chunks
+    assert sw(None, Bp, 2, 2, 64, None) == 1
+    assert sw(A, Bp, 2, 2, 8, None) == 1                                     # chunk < 16 bytes
+    assert sw(A, Bp, 2, 2, 24, None) == 2                                    # chunk % 16
+    assert sw(A + 8, Bp, 2, 2, 64, None) == 3
+    assert sw(A, A + 64, 2, 2, 64, None) == 1                                # dst overlaps src
+
+
+def test_na3d_validation(lib):
+    na = lib.lib.dit_na3d_fwd
+    assert na(None, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 0.1, None) == 1
+    assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 2, 3, 3, 0.1, None) == 1   # even window
+    assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 5, 3, 0.1, None) == 1   # window > grid
+    assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 96, 3, 3, 3, 0.1, None) == 2   # D
+    assert na(A + 8, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 0.1, None) == 3
+    assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 0.0, None) == 1   # scale
+
+
+def test_parts_validation(lib):
+    vp = ctypes.c_void_p
+    arr = lambda *xs: (vp * len(xs))(*xs)
+    pf = lib.lib.dit_attn_fwd_parts
+    q2, k2, v2, o2 = arr(A, A + (1 << 28)), arr(Bp, Bp + (1 << 28)), arr(Cp, Cp + (1 << 28)), arr(O, O + (1 << 28))
+    assert pf(q2, 0, k2, v2, 2, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1          # no query blocks
+    assert pf(q2, 2, k2, v2, 9, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1          # too many blocks
+    assert pf(q2, 2, k2, v2, 2, o2, None, 1, 4, 0, 2, 192, 128, 0.1, None) == 2          # 192 rows per block
+    assert pf(q2, 2, k2, v2, 2, o2, None, 1, 4, 3, 2, 256, 128, 0.1, None) == 1          # heads past part_H
+    assert pf(arr(A, None), 2, k2, v2, 2, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1
+    assert pf(arr(A + 8, A + (1 << 28)), 2, k2, v2, 2, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 3
+    assert pf(q2, 2, k2, v2, 2, arr(O, A), None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1   # out overlaps q
+
+
+def test_acc_and_ipc_validation(lib):
+    acc = lib.lib.dit_attn_fwd_chunk_acc
+    assert acc(A, Bp, Cp, None, L, 1, 2, 256, 256, 64, 0, 256, 0.125, 0, None, None) == 1
+    init = lib.lib.dit_attn_acc_init
+    assert init(O, L, 1, 2, 256, 96, None) == 2
+    assert init(O + 4, L, 1, 2, 256, 64, None) == 3
+    off = ctypes.c_longlong(0)
+    assert lib.lib.dit_ipc_export(None, ctypes.create_string_buffer(64), ctypes.byref(off)) == 1
+    p, b = ctypes.c_void_p(), ctypes.c_void_p()
+    assert lib.lib.dit_ipc_import(None, 0, ctypes.byref(p), ctypes.byref(b)) == 1
+    assert lib.lib.dit_ipc_import(ctypes.create_string_buffer(64), -1, ctypes.byref(p), ctypes.byref(b)) == 1
+    assert lib.lib.dit_ipc_close(None) == 1
