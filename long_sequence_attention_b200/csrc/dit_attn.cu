@@ -145,15 +145,15 @@ int ensure_smem_attr(K kernel, int bytes, std::atomic<uint64_t>& done_mask) {
 template <int D, bool FP8, bool NA, bool PARTS>
 int check_register_split() {
   using C = AttnCfg<D, FP8>;
-  static std::atomic<int> verdict{0};   // 0 unknown, 1 ok, 2 bad
-  int v = verdict.load();
+  static std::atomic<int> split_state{0};   // 0 unknown, 1 ok, 2 bad
+  int v = split_state.load();
   if (v == 0) {
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, attn_fwd_kernel<D, FP8, NA, PARTS>) != cudaSuccess) return DIT_ERR_CUDA;
     const long long launched = static_cast<long long>(attr.numRegs) * C::kThreads;
     const long long wanted = 2LL * 128 * C::kRegsSoftmax + 128LL * C::kRegsCtl;
     v = (attr.numRegs == C::kRegsLaunch && launched >= wanted) ? 1 : 2;
-    verdict.store(v);
+    split_state.store(v);
   }
   return v == 1 ? DIT_OK : DIT_ERR_UNSUPPORTED;
 }
