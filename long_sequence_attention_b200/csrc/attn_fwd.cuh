@@ -181,14 +181,16 @@ __device__ __forceinline__ void apply_mask128(uint32_t (&s)[128], const uint32_t
     if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xFF800000u;
 }
 
-// exp2 on the FMA pipe for x <= 2^7, two values at once with packed fp32x2 instructions:
-// x = n + f with n = rint(x), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (minimax in
-// relative error, max 7.5e-5; coefficients from fit_exp2_poly.py); 2^n by adding n to the
-// exponent field.  x is clamped at -125 so the exponent never underflows (2^-125 stands in
-// for 0; it only ever multiplies V values).  Adding 1.5 * 2^23 rounds x to an integer whose
-// low bits (two's complement) are n; shifting them into the exponent field adds n.
+// exp2 on the FMA pipe, two values at once with packed fp32x2 instructions: x = n + f with
+// n = rint(x), f in [-1/2, 1/2]; 2^f by a degree-3 polynomial (minimax in relative error,
+// max 7.5e-5; coefficients from fit_exp2_poly.py); 2^n by adding n to the exponent field.
+// x is clamped to [-125, 126] so the exponent field neither underflows nor runs into the
+// sign bit: 2^-125 stands in for 0 (it only ever multiplies V values), and any x above 126
+// gives about 2^126, far above every row-sum bound, so a speculative tile whose scores rose
+// that far is always redone exactly.  Adding 1.5 * 2^23 rounds x to an integer whose low
+// bits (two's complement) are n; shifting them into the exponent field adds n.
 __device__ __forceinline__ void exp2_fma2(float x0, float x1, float& e0, float& e1) {
-  const uint64_t x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t x = f2_pack(fminf(fmaxf(x0, -125.0f), 126.0f), fminf(fmaxf(x1, -125.0f), 126.0f));
   const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
   const uint64_t t = f2_add(x, magic);
   const uint64_t f = f2_sub(x, f2_sub(t, magic));
@@ -235,11 +237,7 @@ struct AttnCfg {
   static constexpr int kPWordsHalf = FP8 ? 16 : 32;     // 32-bit P words per half row
   // exp2 split: of every 8 column pairs, this many use the FMA-pipe polynomial (measured
   // best: none at bf16 D=128, 1 at bf16 D=64, 2 for e4m3)
-#ifdef DIT_EMU_PER8
-  static constexpr int kEmuPer8 = DIT_EMU_PER8;
-#else
   static constexpr int kEmuPer8 = FP8 ? 2 : (D == 64 ? 1 : 0);
-#endif
   // bf16: exponentiate with the running max first and redo a tile exactly only when its row
   // sum exceeds kSumBound.  e4m3 P is shifted up by 2^kPShift, so its sums sit near the bound
   // and it always takes the max first.

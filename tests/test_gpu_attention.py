@@ -89,6 +89,34 @@ def test_rising_scores_force_rescaling(cuda_lib, D):
     _check_full(cuda_lib, host, dev, 1.0 / np.sqrt(D), "rising scores")
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_dominant_key_far_above_running_max(cuda_lib, D):
+    """A key in a later KV tile whose score beats the running max of the earlier tiles by
+    about 180 log2 units, in the columns the FMA-pipe exp2 serves at D = 64 (tile 1 column 0,
+    tile 2 column 16).  The speculative softmax must notice the rise and redo the tile
+    exactly; the oracle's result is that key's V row for the aligned query rows."""
+    from workloads import bf16_round
+    S, H = 512, 2
+    scale = 1.0 / np.sqrt(D)
+    q, _ = normal_bf16((1, H, S, D), 41)
+    k, _ = normal_bf16((1, H, S, D), 42)
+    v, vb = normal_bf16((1, H, S, D), 43)
+    u, _ = normal_bf16((D,), 44)
+    gap_raw = 180.0 / (scale * np.log2(np.e))             # 180 log2 units above ~0
+    alpha = np.float32(gap_raw / np.linalg.norm(u.astype(np.float64)))
+    q[:, :, 0:256] = u                                     # both Q tiles of the first unit
+    k[:, 0, 128] = alpha * u / np.linalg.norm(u)           # head 0: tile 1, column 0
+    k[:, 1, 272] = alpha * u / np.linalg.norm(u)           # head 1: tile 2, column 16
+    q, qb = bf16_round(q)
+    k, kb = bf16_round(k)
+    host = (q, k, v)
+    dev = (to_dev_bf16(qb), to_dev_bf16(kb), to_dev_bf16(vb))
+    out, _ = _check_full(cuda_lib, host, dev, scale, f"dominant key D={D}")
+    o = host_f64(out)
+    assert np.max(np.abs(o[0, 0, :256] - v[0, 0, 128].astype(np.float64))) <= 2e-2
+    assert np.max(np.abs(o[0, 1, :256] - v[0, 1, 272].astype(np.float64))) <= 2e-2
+
+
 @pytest.mark.parametrize("scale", [1e-3, 0.05, 0.5])
 def test_scale_range(cuda_lib, scale):
     host, dev = _case(1, 2, 520, 520, 128, seed=int(scale * 1000) + 5, std=2.0)
