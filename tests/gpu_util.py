@@ -38,6 +38,15 @@ def metrics(out_gpu: np.ndarray, out_ref: np.ndarray, lse_gpu=None, lse_ref=None
     return m
 
 
+def assert_fp8_parity(m, what=""):
+    """FP8-E4M3 inputs: rel-L2 against the oracle on the dequantised inputs, and the same LSE
+    bar as bf16 (the row sums are formed in fp32 before P is rounded to E4M3, so the LSE
+    carries no FP8 rounding)."""
+    assert m["rel_l2"] <= FP8_REL_L2, (what, m)
+    assert "lse_max_abs" in m, (what, "FP8 parity needs the LSE compared too")
+    assert m["lse_max_abs"] <= LSE_MAX_ABS, (what, m)
+
+
 def assert_bf16_parity(m, what=""):
     assert m["rel_l2"] <= BF16_REL_L2, (what, m)
     assert m["max_abs"] <= BF16_MAX_ABS, (what, m)

@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 from oracle import fp8 as ofp8
-from gpu_util import FP8_REL_L2, host_f64, metrics, to_dev_bf16
+from gpu_util import assert_fp8_parity, host_f64, metrics, to_dev_bf16
 from workloads import WORKLOADS, make_qkv, normal_bf16, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -66,8 +66,7 @@ def test_block_fp8_attention_matches_oracle(cuda_lib, Sq, Skv):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(*deq, scale)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
-    assert m["lse_max_abs"] <= 1e-2, m
+    assert_fp8_parity(m)
 
 
 @pytest.mark.parametrize("k0,k1", [(0, 700), (256, 700), (128, 129), (640, 700)])
@@ -79,7 +78,7 @@ def test_block_fp8_chunk_fp32(cuda_lib, k0, k1):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(deq[0], deq[1][:, :, k0:k1], deq[2][:, :, k0:k1], scale)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
 
 
 def test_block_fp8_all_zero_v_block(cuda_lib):
@@ -98,7 +97,7 @@ def test_block_fp8_all_zero_v_block(cuda_lib):
     rc, rd = ofp8.quantize_per_block(x)
     ro, rl = oracle.attention(deq[0], deq[1], ofp8.dequantize_per_block(rc, rd), 0.1)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
 
 
 def test_block_scales_beat_per_tensor_on_uneven_heads(cuda_lib):
@@ -150,7 +149,7 @@ def test_block_fp8_video_sampled_rows(cuda_lib):
     og = host_f64(out[:, heads][:, :, rows])
     lg = lse[:, heads][:, :, rows].cpu().numpy().astype(np.float64)
     m = metrics(og, ro, lg, rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
 
 
 def test_block_fp8_argument_checks(cuda_lib):

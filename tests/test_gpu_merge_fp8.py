@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from oracle import fp8 as ofp8
-from gpu_util import FP8_REL_L2, assert_bf16_parity, host_f64, metrics, to_dev_bf16, to_dev_u8
+from gpu_util import assert_fp8_parity, assert_bf16_parity, host_f64, metrics, to_dev_bf16, to_dev_u8
 from workloads import WORKLOADS, make_qkv, normal_bf16, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -150,8 +150,7 @@ def test_fp8_attention_small(cuda_lib, S):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(*deq, scale)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
-    assert m["lse_max_abs"] <= 1e-2, m
+    assert_fp8_parity(m)
 
 
 def test_fp8_chunk_and_merge(cuda_lib):
@@ -165,7 +164,7 @@ def test_fp8_chunk_and_merge(cuda_lib):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(*deq, scale)
     m = metrics(host_f64(mo), ro, ml.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
 
 
 def test_fp8_video_sampled_rows(cuda_lib):
@@ -199,7 +198,7 @@ def test_fp8_video_sampled_rows(cuda_lib):
     og = host_f64(out[:, heads][:, :, rows])
     lg = lse[:, heads][:, :, rows].cpu().numpy().astype(np.float64)
     m = metrics(og, ro, lg, rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
     # for context: error against the bf16-input oracle
     rb, _ = oracle.attention(d["q"][:, heads], d["k"][:, heads], d["v"][:, heads], w.scale, rows=rows)
     print("fp8 video vs dequantised oracle", m, "vs bf16 oracle rel_l2",

@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from oracle import fp8 as ofp8
-from gpu_util import FP8_REL_L2, assert_bf16_parity, host_f64, metrics, to_dev_bf16
+from gpu_util import assert_fp8_parity, assert_bf16_parity, host_f64, metrics, to_dev_bf16
 from workloads import WORKLOADS, chunk_bounds, make_qkv, normal_bf16, sample_rows
 
 pytestmark = pytest.mark.gpu
@@ -67,7 +67,7 @@ def test_fp8_ring_accumulate(cuda_lib):
     torch.cuda.synchronize()
     ro, rl = oracle.attention(*deq, scale)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
-    assert m["rel_l2"] <= FP8_REL_L2, m
+    assert_fp8_parity(m)
 
 
 def test_flux2048_four_fused_ring_steps_sampled_rows(cuda_lib):

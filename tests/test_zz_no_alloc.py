@@ -5,7 +5,8 @@ while capturing a CUDA graph, or under a framework allocator that forbids raw cu
 so they cannot provide the workspace dit_quant_fp8 needs.  dit_quant_fp8_noalloc keeps its
 scratch in a static array inside the library instead.  This test calls it through the C ABI
 twice in a row, on inputs of different sizes and ranges (so stale scratch from the first call
-would show up in the second), and checks both results against the workspace entry point:
+would show up in the second), and checks both results against the workspace entry point and
+against the oracle's own quantiser (so a fault shared by both CUDA quantisers cannot pass):
 E4M3 codes and descale are byte work, so the tolerance is exact equality.
 
 The file is named to be collected last: it must pass on its own in a fresh process (where its
@@ -18,6 +19,7 @@ import numpy as np
 import pytest
 
 from gpu_util import to_dev_bf16
+from oracle import fp8 as ofp8
 from workloads import normal_bf16
 
 pytestmark = pytest.mark.gpu
@@ -50,13 +52,16 @@ def test_no_alloc_quant_matches_workspace_entry_point_on_two_calls(cuda_lib):
     # call 1: many blocks and a large range; call 2: fewer blocks and a small range
     cases = [((1 << 22) + 5, 4.0, 301), ((1 << 16) + 3, 0.25, 302)]
     for n, std, seed in cases:
-        _, bits = normal_bf16((n,), seed, std=std)
+        host, bits = normal_bf16((n,), seed, std=std)
         x = to_dev_bf16(bits)
         ref_codes, ref_descale = _with_workspace(cuda_lib, x, n)
         codes, descale = _no_alloc_via_c_abi(cuda_lib, x, n)
         torch.cuda.synchronize()
         assert torch.equal(descale, ref_descale), (n, descale.item(), ref_descale.item())
         assert torch.equal(codes, ref_codes), n
+        oracle_codes, oracle_descale = ofp8.quantize_per_tensor(host)
+        assert np.float32(descale.item()) == oracle_descale, (n, descale.item(), oracle_descale)
+        assert np.array_equal(codes.cpu().numpy(), oracle_codes), n
     assert cuda_lib.dit_device_status(clear=True) == 0
 
 
