@@ -496,6 +496,21 @@ int dit_attn_fwd_parts(const void* const* q_parts, int n_q_parts, const void* co
           overlaps(out_parts[i], part_bytes, v_parts[j], part_bytes))
         return DIT_ERR_INVALID_ARG;
   }
+  // An LSE block must not overlap any input or output block, nor another LSE block: the
+  // kernel's LSE stores would otherwise race with TMA loads of the same bytes.
+  const size_t lse_bytes = static_cast<size_t>(B) * part_H * part_rows * 4;
+  if (lse_parts != nullptr) {
+    for (int i = 0; i < n_q_parts; ++i) {
+      const void* l = lse_parts[i];
+      for (int j = 0; j < n_q_parts; ++j)
+        if (overlaps(l, lse_bytes, q_parts[j], part_bytes) || overlaps(l, lse_bytes, out_parts[j], part_bytes) ||
+            (i != j && overlaps(l, lse_bytes, lse_parts[j], lse_bytes)))
+          return DIT_ERR_INVALID_ARG;
+      for (int j = 0; j < n_kv_parts; ++j)
+        if (overlaps(l, lse_bytes, k_parts[j], part_bytes) || overlaps(l, lse_bytes, v_parts[j], part_bytes))
+          return DIT_ERR_INVALID_ARG;
+    }
+  }
   AttnParams prm;
   std::memset(&prm, 0, sizeof(prm));
   prm.B = B; prm.H = H; prm.S_q = static_cast<int>(S_q); prm.S_kv = static_cast<int>(S_kv);

@@ -185,6 +185,13 @@ def test_parts_validation(lib):
     assert pf(arr(A, None), 2, k2, v2, 2, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1
     assert pf(arr(A + 8, A + (1 << 28)), 2, k2, v2, 2, o2, None, 1, 4, 0, 2, 256, 128, 0.1, None) == 3
     assert pf(q2, 2, k2, v2, 2, arr(O, A), None, 1, 4, 0, 2, 256, 128, 0.1, None) == 1   # out overlaps q
+    fp = ctypes.c_void_p
+    larr = lambda *xs: (fp * len(xs))(*xs)
+    assert pf(q2, 2, k2, v2, 2, o2, larr(L, A), 1, 4, 0, 2, 256, 128, 0.1, None) == 1          # lse overlaps q
+    assert pf(q2, 2, k2, v2, 2, o2, larr(L, Bp + 64), 1, 4, 0, 2, 256, 128, 0.1, None) == 1    # lse overlaps k
+    assert pf(q2, 2, k2, v2, 2, o2, larr(L, Cp), 1, 4, 0, 2, 256, 128, 0.1, None) == 1         # lse overlaps v
+    assert pf(q2, 2, k2, v2, 2, o2, larr(L, O + 256), 1, 4, 0, 2, 256, 128, 0.1, None) == 1    # lse overlaps out
+    assert pf(q2, 2, k2, v2, 2, o2, larr(L, L + 64), 1, 4, 0, 2, 256, 128, 0.1, None) == 1     # lse blocks overlap
 
 
 def test_acc_and_ipc_validation(lib):
