@@ -42,7 +42,9 @@ from workloads import WORKLOADS, chunk_bounds, make_qkv  # noqa: E402
 METRIC = "DiT attention TFLOP/s (4·B·H·S²·D) and % of B200 dense BF16/FP8 peak, 1 GPU"
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_fwd_bf16_flux2048.txt")
 KERNEL_SRC = os.path.join(ROOT, "long_sequence_attention_b200", "csrc", "attn_fwd.cuh")
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# used only when MEASURED_PEAKS.json is absent: an earlier B200 measurement (HBM
+# copy, burst cuBLAS bf16); there is no fallback for the sustained figure
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
 
 # ----------------------------------------------------------------------------- helpers
