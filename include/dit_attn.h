@@ -276,7 +276,9 @@ int dit_attn_fwd_fp8_blocks(const void* q8, const void* k8, const void* v8, cons
  *   rejected with DIT_ERR_UNSUPPORTED.
  *   Set-up: the first call on each device (with that device current) looks up the array's
  *   device address with cudaGetSymbolAddress; make that first call before any stream
- *   capture.  Later calls reuse the address.
+ *   capture.  Later calls reuse the address while the device keeps the same context; after
+ *   a cudaDeviceReset the next call repeats the set-up (the reset reloads the module), so
+ *   that call, too, should come before any capture.
  *   Sharing: all calls on a device share the one array and it keeps the last call's
  *   contents.  Nothing in it needs to start at zero (each call writes every slot it reads
  *   before reading it), but calls whose kernels overlap on the GPU (different streams, no

@@ -283,17 +283,46 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
 float* g_noalloc_scratch_ptr[kMaxDevices] = {};
+CUcontext g_noalloc_ctx[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (set-up on first use per device).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+// cuCtxGetCurrent through the runtime's driver entry-point lookup (no libcuda link).
+CtxGetCurrentFn ctx_current_fn() {
+  static std::once_flag once;
+  static CtxGetCurrentFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the static scratch on the current device.  Set-up happens on the first
+// call per device, and again if the device's context has changed since (a cudaDeviceReset
+// reloads the module, which may move the array): the cached address belongs to the context
+// it was looked up in.
 int noalloc_scratch(float** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return DIT_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return DIT_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_scratch_ptr[dev] == nullptr) {
+  CUcontext ctx = nullptr;
+  CtxGetCurrentFn cur = ctx_current_fn();
+  if (g_noalloc_scratch_ptr[dev] != nullptr) {
+    // the runtime has made the device's context current by now (cudaGetDevice does not, so
+    // ask the driver only when there is a cached address to validate)
+    if (cur == nullptr || cur(&ctx) != CUDA_SUCCESS) return DIT_ERR_CUDA;
+  }
+  if (g_noalloc_scratch_ptr[dev] == nullptr || ctx != g_noalloc_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_quant_noalloc_scratch) != cudaSuccess || p == nullptr) return DIT_ERR_CUDA;
+    if (cur == nullptr || cur(&ctx) != CUDA_SUCCESS) return DIT_ERR_CUDA;
     g_noalloc_scratch_ptr[dev] = static_cast<float*>(p);
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_scratch_ptr[dev];
   return DIT_OK;
