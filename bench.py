@@ -1,6 +1,7 @@
 """Benchmark of the DiT joint-attention hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload flux_2048] [--impl ours|reference]
+                    [--mode replicas|ring|ring_peers|ulysses|ulysses_peers]
 
 One step = one pass of the whole hot path over one batch of synthetic input of the chosen
 workload (default: FLUX-2048-like joint attention, B=1 H=24 S=16896 D=128, bf16):
@@ -14,6 +15,12 @@ pass each count once), whole job, max over ranks.  Inputs (Q, K, V) are resident
 larger than the 126 MB L2, so no L2 flush is needed between steps.  Multi-GPU (torchrun):
 every rank runs its own replica batch (independent problems; no data-path collective),
 scaling "weak".
+
+--mode ring|ring_peers|ulysses|ulysses_peers instead splits ONE sequence of the workload
+across the ranks by a sequence-parallel form of the xDiT overview page (section 3.2.2): the
+KV ring over NCCL with fused ring steps, the ring without a ring over peer memory, the
+Ulysses all-to-all over NCCL, or Ulysses fused over peer memory.  A step is one attention over
+the whole sequence; value = its FLOPs / max-over-ranks time, scaling "strong".
 
 --impl reference times the fp64 CPU oracle (the only other implementation of this path) on
 the host cores, on a bounded sample of the same workload per step.
@@ -294,6 +301,186 @@ class Step:
                 ev[5].record(stream)
 
 
+SEQPAR_MODES = ("ring", "ring_peers", "ulysses", "ulysses_peers")
+
+
+def seqpar_blocks(mode: str, S: int, H: int, P: int):
+    """Rows [a, b) of the sequence each of P ranks holds in a sequence-parallel mode, or a
+    one-line reason why the split is not supported.  The NCCL ring takes any split (the last
+    rank gets the remainder); the peer-memory ring and both Ulysses forms need S/P rows per
+    rank, a multiple of 128 when P > 1 (a 128-row tile must not straddle two ranks), and
+    Ulysses needs H divisible by P."""
+    if mode == "ring":
+        return chunk_bounds(S, P), None
+    if S % P != 0 or (P > 1 and (S // P) % 128 != 0):
+        return None, f"{mode} needs S/P rows per rank, a multiple of 128 (S={S}, P={P})"
+    if mode in ("ulysses", "ulysses_peers") and H % P != 0:
+        return None, f"{mode} needs H divisible by P (H={H}, P={P})"
+    if mode in ("ring_peers", "ulysses_peers") and P > 8:
+        return None, f"{mode} reads at most 8 ranks' blocks"
+    n = S // P
+    return [(r * n, (r + 1) * n) for r in range(P)], None
+
+
+def seqpar_launches(mode: str, B: int, P: int) -> int:
+    """Library kernel launches of one sequence-parallel step on one rank."""
+    if mode == "ring":
+        return 1 + P + 1                    # accumulator init, P fused ring steps, bf16 finish
+    if mode == "ulysses":
+        return 1 + (5 if (B > 1 and P > 1) else 0)   # attention (+ layout swaps at B > 1)
+    return 1                                # one fused multi-block launch
+
+
+def run_seqpar(args, rank, local_rank, world):
+    """One attention over the workload's whole sequence, split across the ranks by a USP
+    dimension (xDiT overview, section 3.2.2): each rank holds a block of rows of Q, K, V and
+    gets its rows of O and LSE.  value = the one attention's FLOPs per step / max-over-ranks
+    time (strong scaling: the total work is fixed as ranks are added)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    if rank == 0 or world == 1:
+        ensure_library()
+    if world > 1:
+        deadline = time.time() + 900
+        lib = os.path.join(ROOT, "long_sequence_attention_b200", "libdit_attn.so")
+        while not os.path.exists(lib) and time.time() < deadline:
+            time.sleep(1.0)
+    import long_sequence_attention_b200 as lsa
+    from long_sequence_attention_b200 import ring as lring
+    from long_sequence_attention_b200 import ulysses as lul
+
+    w = WORKLOADS[args.workload]
+    B, H, S, D = w.B, w.H, w.S, w.D
+    blocks, why = seqpar_blocks(args.mode, S, H, world)
+    if why is not None:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "mode": args.mode, "n_gpus": world, "unavailable": why}), flush=True)
+        return
+    dev = torch.device(f"cuda:{local_rank}")
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    else:
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=30))
+        dist.init_process_group("nccl", store=store, rank=0, world_size=1, timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    ranks = Ranks(world, "nccl", dev)
+
+    data = make_qkv(w)                      # one sequence, the same on every rank; each keeps its rows
+    a, b = blocks[rank]
+    to_dev = lambda name: torch.from_numpy(np.ascontiguousarray(data[name + "_bits"][:, :, a:b]).view(np.int16)) \
+        .view(torch.bfloat16).to(dev)
+    q, k, v = to_dev("q"), to_dev("k"), to_dev("v")
+    peer_ops = lul.CudaPeerOps() if args.mode in ("ring_peers", "ulysses_peers") else None
+    out_buf = torch.empty_like(q)
+    lse_buf = torch.empty((B, H, b - a), dtype=torch.float32, device=dev)
+
+    def step():
+        if args.mode == "ring":
+            return lring.ring_attention_dist(q, k, v, w.scale, out_dtype=torch.bfloat16, block_lens=[y - x for x, y in blocks])
+        if args.mode == "ring_peers":
+            return lring.ring_attention_peers(q, k, v, w.scale, ops=peer_ops, out=out_buf, lse=lse_buf)
+        if args.mode == "ulysses":
+            return lul.ulysses_attention_dist(q, k, v, w.scale)
+        return lul.ulysses_attention_peers(q, k, v, w.scale, ops=peer_ops, out=out_buf, lse=lse_buf)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if lsa.dit_device_status(clear=True) != 0:
+        raise RuntimeError("device status after warm-up is not OK")
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(smi_device_id(dev)) as clk:
+        t0.record()
+        for _ in range(args.steps):
+            o, l = step()
+        t1.record()
+        torch.cuda.synchronize()
+    dist.barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = ranks.max(t0.elapsed_time(t1))
+    status = lsa.dit_device_status(clear=True)
+
+    # this rank's rows against a local forward over the whole sequence (one launch)
+    kf, vf = (torch.from_numpy(data[n + "_bits"].view(np.int16)).view(torch.bfloat16).to(dev) for n in "kv")
+    ref_o = torch.empty((B, H, b - a, D), dtype=torch.float32, device=dev)
+    ref_l = torch.empty((B, H, b - a), dtype=torch.float32, device=dev)
+    qs = q.contiguous()
+    lsa.dit_attn_fwd_chunk(qs, kf, vf, ref_o, ref_l, B, H, b - a, S, D, 0, S, w.scale, lsa.DIT_BF16, lsa.DIT_FP32)
+    torch.cuda.synchronize()
+    diff = ranks.max(float((o.float() - ref_o).abs().max().item()))
+    ldiff = ranks.max(float((l - ref_l).abs().max().item()))
+    del kf, vf, ref_o, ref_l
+
+    # end to end: this rank's rows copied in from pinned host memory and its O/LSE copied back
+    host_in = [torch.from_numpy(np.ascontiguousarray(data[n + "_bits"][:, :, a:b]).view(np.int16))
+               .view(torch.bfloat16).pin_memory() for n in "qkv"]
+    host_o = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    host_l = torch.empty((B, H, b - a), dtype=torch.float32).pin_memory()
+    n_e2e = max(3, min(args.steps, 10))
+
+    def e2e_step():
+        for h, d_ in zip(host_in, (q, k, v)):
+            d_.copy_(h, non_blocking=True)
+        o_, l_ = step()
+        host_o.copy_(o_, non_blocking=True)
+        host_l.copy_(l_, non_blocking=True)
+    e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = ranks.max(e0.elapsed_time(e1)) / n_e2e
+    if peer_ops is not None:
+        dist.barrier()
+        peer_ops.close()
+    dist.barrier()
+    dist.destroy_process_group()
+    if rank != 0:
+        return
+    peaks, peaks_src = load_peaks()
+    ms = elapsed_ms / args.steps
+    value = w.flops / (ms * 1e-3) / 1e12
+    per_gpu = value / world
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) rounded to bf16; no weights involved)",
+        "config": {"workload": w.name, "B": B, "H": H, "S": S, "D": D, "scale": w.scale,
+                   "step": {"ring": "ring_attention_dist (NCCL send/recv + dit_attn_fwd_chunk_acc)",
+                            "ring_peers": "ring_attention_peers (dit_attn_fwd_parts over peer memory)",
+                            "ulysses": "ulysses_attention_dist (NCCL all-to-all + dit_attn_fwd_seg)",
+                            "ulysses_peers": "ulysses_attention_peers (dit_attn_fwd_parts over peer memory)"}[args.mode],
+                   "rows_per_rank": [y - x for x, y in blocks],
+                   "l2": "no flush: Q/K/V exceed the 126 MB L2" if 3 * B * H * S * D * 2 > 126e6 else "inputs fit in L2",
+                   "parallelism": f"{args.mode}{world}"},
+        "roofline": {"bound": "tensor", "kernel": args.mode + " step, per GPU", "achieved": round(per_gpu, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(per_gpu / peaks["bf16_tflops"], 4),
+                     "peak_source": f"{peaks_src} bf16_tflops (burst)", "traffic": None},
+        "gpu_launches": seqpar_launches(args.mode, B, world) * args.steps,
+        "device_status": status,
+        "max_abs_vs_single_launch": diff, "lse_max_abs_vs_single_launch": ldiff,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(w.flops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 3),
+                "steps": n_e2e, "h2d_bytes_per_step": sum(h.numel() * h.element_size() for h in host_in) * world,
+                "d2h_bytes_per_step": (host_o.numel() * 2 + host_l.numel() * 4) * world},
+    }
+    if world == 1 and not args.skip_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
 def ensure_library():
     """Build the in-tree CUDA library if it is missing or older than its sources (a no-op
     otherwise), without importing the package first."""
@@ -366,6 +553,7 @@ def run_ours(args, rank, local_rank, world):
     seg = run_seg_context(lsa, step, stream, ranks)
     parts = run_parts_context(lsa, step, stream, ranks)
     fp8b = run_fp8_blocks_context(lsa, step, stream, ranks)
+    fwds = run_forwards_context(lsa, dev, stream, ranks) if not args.skip_forwards else None
 
     ranks.close()
     if rank != 0:
@@ -435,6 +623,8 @@ def run_ours(args, rank, local_rank, world):
     if parts is not None:
         line["ulysses_peers_virtual"] = parts
     line["fp8_blocks"] = fp8b
+    if fwds is not None:
+        line["forwards"] = fwds
     line["clocks"] = clk.summary()
     line["e2e"] = e2e
     if world == 1 and not args.skip_cpu_baseline:
@@ -591,6 +781,55 @@ def run_fp8_blocks_context(lsa, step, stream, ranks):
             "fwd_ms": round(ms_f, 4), "fwd_tflops": round(tf, 2),
             "fwd_frac_of_2x_bf16_peak": round(tf / (2 * peaks["bf16_tflops"]), 4),
             "calls": "3 x dit_quant_fp8_blocks, dit_attn_fwd_fp8_blocks"}
+
+
+def run_forwards_context(lsa, dev, stream, ranks, reps: int = 5):
+    """The forward kernel alone on every DiT workload of the suite, beside the step: bf16 on
+    SD3-1024 (D = 64), FLUX-1024, FLUX-2048 and video, and E4M3 with per-tensor scales on
+    FLUX-2048 and video.  Inputs are N(0,1) drawn on the device (timing only; parity of every
+    configuration is covered by the tests).  bf16 against the measured bf16 peak, E4M3 against
+    twice it (the nominal dense FP8 / BF16 ratio)."""
+    import torch
+    peaks, src = load_peaks()
+    g = torch.Generator(device=dev)
+    g.manual_seed(11)
+    res = {}
+    plan = [("sd3_1024", False), ("flux_1024", False), ("flux_2048", False), ("video", False),
+            ("flux_2048", True), ("video", True)]
+    for name, fp8 in plan:
+        w = WORKLOADS[name]
+        B, H, S, D = w.B, w.H, w.S, w.D
+        x = [torch.randn((B, H, S, D), generator=g, device=dev).to(torch.bfloat16) for _ in range(3)]
+        out = torch.empty((B, H, S, D), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=dev)
+        if fp8:
+            n = B * H * S * D
+            codes = [torch.empty((B, H, S, D), dtype=torch.uint8, device=dev) for _ in range(3)]
+            ds = torch.empty((3,), dtype=torch.float32, device=dev)
+            wsb = lsa.dit_quant_fp8_workspace_bytes(n)
+            ws = torch.empty((wsb // 4 + 1,), dtype=torch.float32, device=dev)
+            for i in range(3):
+                lsa.dit_quant_fp8(x[i], codes[i], ds[i:i + 1], n, ws, wsb, stream)
+            del x
+            call = lambda: lsa.dit_attn_fwd(codes[0], codes[1], codes[2], out, lse, B, H, S, D, w.scale,
+                                            lsa.DIT_FP8_E4M3, ds, stream)
+        else:
+            call = lambda: lsa.dit_attn_fwd(x[0], x[1], x[2], out, lse, B, H, S, D, w.scale, lsa.DIT_BF16, None,
+                                            stream)
+        ms = _time_calls(call, stream, ranks, reps)
+        tf = w.flops * ranks.world / (ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+        res[name + ("_e4m3" if fp8 else "_bf16")] = {
+            "B": B, "H": H, "S": S, "D": D, "ms": round(ms, 4), "tflops": round(tf, 2),
+            "frac": round(tf / peak, 4),
+            "peak": round(peak, 1), "peak_source": f"{src} bf16_tflops (burst)" + (" x 2" if fp8 else "")}
+        del out, lse
+        if fp8:
+            del codes, ds, ws
+        else:
+            del x
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_ring_fused(lsa, step, stream, ranks, reps: int = 10):
@@ -796,9 +1035,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="flux_2048", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--mode", default="replicas", choices=("replicas",) + SEQPAR_MODES,
+                    help="replicas: one independent batch per rank (default); ring / ring_peers / ulysses / "
+                         "ulysses_peers: one sequence split across the ranks by that sequence-parallel form")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU work of the oracle baseline sample")
     ap.add_argument("--ref-step-seconds", type=float, default=6.0, help="CPU work per --impl reference step")
     ap.add_argument("--skip-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-forwards", action="store_true",
+                    help="leave out the per-workload forward timings reported beside the step")
     ap.add_argument("--e2e-groups", type=int, default=0,
                     help="head groups of the end-to-end pipeline (copies of one group overlap kernels of another);"
                          " 0 = about one wave of work units per group")
@@ -810,6 +1054,8 @@ def main():
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":
         run_reference(args, rank, world)
+    elif args.mode != "replicas":
+        run_seqpar(args, rank, local_rank, world)
     else:
         run_ours(args, rank, local_rank, world)
 

@@ -79,3 +79,33 @@ def test_reference_arm_under_torchrun_two_ranks():
     assert out.returncode == 0, out.stderr
     lines = _json_lines(out.stdout)
     assert len(lines) == 1 and lines[0]["n_gpus"] == 2      # rank 0 alone prints
+
+
+def test_seqpar_blocks_and_launch_counts():
+    sys.path.insert(0, ROOT)
+    import bench
+    # the NCCL ring takes any split; the last rank gets the remainder
+    blocks, why = bench.seqpar_blocks("ring", 1000, 24, 3)
+    assert why is None and blocks == [(0, 333), (333, 666), (666, 1000)]
+    # FLUX-2048 over 4 ranks: 4224 rows each (33 tiles); over 8 ranks 2112 is not a tile multiple
+    blocks, why = bench.seqpar_blocks("ulysses", 16896, 24, 4)
+    assert why is None and blocks[1] == (4224, 8448)
+    for mode in ("ulysses", "ulysses_peers", "ring_peers"):
+        assert bench.seqpar_blocks(mode, 16896, 24, 8)[1] is not None
+        assert bench.seqpar_blocks(mode, 16896, 24, 1)[0] == [(0, 16896)]
+    assert bench.seqpar_blocks("ulysses", 4096, 24, 16)[1] is not None          # 16 does not divide 24
+    assert bench.seqpar_blocks("ulysses_peers", 16384, 32, 16)[1] is not None    # more than 8 ranks
+    assert bench.seqpar_launches("ring", 1, 4) == 6
+    assert bench.seqpar_launches("ulysses", 2, 4) == 6 and bench.seqpar_launches("ulysses", 1, 4) == 1
+
+
+def test_seqpar_mode_reports_an_unsupported_split():
+    """Under torchrun with two ranks, a split the mode cannot take (S/P not a multiple of 128)
+    prints one 'unavailable' line from rank 0 and exits 0 on every rank before any GPU work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--gpus", "2",
+           "--mode", "ulysses", "--workload", "sd3_1024", "--steps", "3", "--warmup", "3"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr
+    lines = _json_lines(out.stdout)
+    assert len(lines) == 1 and "unavailable" in lines[0] and lines[0]["n_gpus"] == 2

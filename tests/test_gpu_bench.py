@@ -44,3 +44,20 @@ def test_bench_video_e2e_pipeline_matches():
     d = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")][0]
     assert d["e2e"]["head_groups"] == 5 and d["e2e"]["matches_whole_tensor_calls"] is True
     assert d["device_status"] == 0
+
+
+@pytest.mark.parametrize("mode", ["ring", "ring_peers", "ulysses", "ulysses_peers"])
+def test_bench_sequence_parallel_modes_on_one_gpu(mode):
+    """bench.py --mode <form> on one rank (a one-rank NCCL group): the JSON contract, strong
+    scaling, and the rank's rows agreeing with a single launch over the whole sequence."""
+    cmd = [sys.executable, "bench.py", "--mode", mode, "--workload", "sd3_1024", "--steps", "3", "--warmup", "3",
+           "--skip-cpu-baseline"]
+    out = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(l) for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["scaling"] == "strong" and d["config"]["parallelism"] == mode + "1" and d["value"] > 0
+    assert d["device_status"] == 0 and d["gpu_launches"] > 0
+    assert d["max_abs_vs_single_launch"] <= 2e-2 and d["lse_max_abs_vs_single_launch"] <= 1e-3
+    assert d["e2e"]["h2d_bytes_per_step"] == 3 * 2 * 24 * 4429 * 64 * 2
