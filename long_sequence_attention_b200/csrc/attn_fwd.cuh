@@ -235,9 +235,10 @@ struct AttnCfg {
   static constexpr float kPShift = FP8 ? 4.0f : 0.0f;
   static constexpr float kSumBound = 256.0f;           // = 2^(kRescaleLog2 + kPShift)
   static constexpr int kPWordsHalf = FP8 ? 16 : 32;     // 32-bit P words per half row
-  // exp2 split: of every 8 column pairs, this many use the FMA-pipe polynomial (measured
-  // best: none at bf16 D=128, 1 at bf16 D=64, 2 for e4m3)
-  static constexpr int kEmuPer8 = FP8 ? 2 : (D == 64 ? 1 : 0);
+  // exp2 split: bit i set = column pair i of every 8 uses the FMA-pipe polynomial instead of
+  // the MUFU (measured best: none at bf16 D=128; pairs 3 and 7 at bf16 D=64 and for e4m3,
+  // spread out so the polynomial's FMA work falls between MUFU instructions)
+  static constexpr int kEmuMask = (FP8 || D == 64) ? 0x88 : 0x00;
   // bf16: exponentiate with the running max first and redo a tile exactly only when its row
   // sum exceeds kSumBound.  e4m3 P is shifted up by 2^kPShift, so its sums sit near the bound
   // and it always takes the max first.
@@ -279,10 +280,10 @@ __device__ __forceinline__ float row_max128(const uint32_t (&s)[128]) {
   return fmax3(fmax3(mx[0], mx[1], mx[2]), fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
 }
 
-// p = 2^(cl*s - mc) for the 128 scores of a row, two lanes per instruction; of every 8
-// column pairs, kEmu use the FMA-pipe polynomial and the rest the MUFU ex2.  Writes the P
-// words (bf16 pairs: 64 words, or e4m3 quads: 32 words) and the row sum.
-template <bool FP8, int kEmu>
+// p = 2^(cl*s - mc) for the 128 scores of a row, two lanes per instruction; column pair c
+// uses the FMA-pipe polynomial when bit c % 8 of kEmuMask is set, the MUFU ex2 otherwise.
+// Writes the P words (bf16 pairs: 64 words, or e4m3 quads: 32 words) and the row sum.
+template <bool FP8, int kEmuMask>
 __device__ __forceinline__ void exp_pass(const uint32_t (&s)[128], float cl, float mc, uint32_t* pw, float& sum) {
   const uint64_t cl2 = f2_pack(cl, cl), nmc2 = f2_pack(-mc, -mc);
   uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
@@ -291,7 +292,7 @@ __device__ __forceinline__ void exp_pass(const uint32_t (&s)[128], float cl, flo
     const uint64_t x = f2_fma(f2_pack(__uint_as_float(s[2 * c2]), __uint_as_float(s[2 * c2 + 1])), cl2, nmc2);
     float x0, x1, e0, e1;
     f2_unpack(x, x0, x1);
-    if ((c2 & 7) < kEmu) {
+    if ((kEmuMask >> (c2 & 7)) & 1) {
       exp2_fma2(x0, x1, e0, e1);
     } else {
       e0 = ex2_approx(x0);
@@ -680,7 +681,7 @@ __global__ void __launch_bounds__(384, 1)
       // (NA: a row whose window has missed every tile so far has no max yet: exact route)
       bool slow = (j == 0) || !C::kSpeculative || (NA && __any_sync(0xffffffffu, m_use == -INFINITY));
       if (!slow) {
-        exp_pass<FP8, C::kEmuPer8>(s, cl, m_use * cl - C::kPShift, pw, sum);
+        exp_pass<FP8, C::kEmuMask>(s, cl, m_use * cl - C::kPShift, pw, sum);
         slow = __any_sync(0xffffffffu, !(sum <= C::kSumBound));
       }
       if (slow) {
@@ -699,7 +700,7 @@ __global__ void __launch_bounds__(384, 1)
             alpha = ex2_approx(m_use - m_new);               // 0 when m_use = -inf
             m_use = m_new;
           }
-          exp_pass<FP8, C::kEmuPer8>(s, clj, m_use - C::kPShift - lrj, pw, sum);
+          exp_pass<FP8, C::kEmuMask>(s, clj, m_use - C::kPShift - lrj, pw, sum);
           sum *= inv_rj;
         } else {
           const float m_new = fmaxf(m_use, row_max128(s));
@@ -710,7 +711,7 @@ __global__ void __launch_bounds__(384, 1)
           }
           // (a row with no key in its window yet keeps m_use = -inf: exponents of -inf, p = 0)
           const float mc = (NA && m_use == -INFINITY) ? 0.0f : m_use * cl;
-          exp_pass<FP8, C::kEmuPer8>(s, cl, mc - C::kPShift, pw, sum);
+          exp_pass<FP8, C::kEmuMask>(s, cl, mc - C::kPShift, pw, sum);
         }
       }
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
