@@ -149,14 +149,48 @@ REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_pow
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples (every 200 ms) during the timed region."""
+    """SM clock and throttle-reason samples during the timed region: through NVML every 10 ms
+    when the bindings load (reading only; nothing is set), else nvidia-smi every 100 ms."""
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index):
         self.dev = device_index
         self.proc = None
         self.lines = []
+        self.nvml = None
+        self.stop = threading.Event()
+
+    def _nvml_sample(self, nv, handle):
+        sm = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+        mx = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+        bits = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+        self.lines.append(f"{sm}, {mx}, 0, {bits:#x}")
+
+    def _nvml_loop(self, nv, handle):
+        while not self.stop.is_set():
+            try:
+                self._nvml_sample(nv, handle)
+            except Exception:
+                return
+            self.stop.wait(0.01)
 
     def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            dev = str(self.dev)
+            handle = (nv.nvmlDeviceGetHandleByUUID(dev) if dev.startswith("GPU-")
+                      else nv.nvmlDeviceGetHandleByIndex(int(dev)))
+            self.nvml = nv
+            self.handle = handle
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, handle), daemon=True)
+            self.thread.start()
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 2.0:
+                time.sleep(0.005)
+            self.lines.clear()
+            return self
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev),
@@ -178,6 +212,17 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *exc):
+        if self.nvml is not None:
+            self.stop.set()
+            self.thread.join(timeout=2)
+            try:
+                self._nvml_sample(self.nvml, self.handle)   # one at the end: short regions get one too
+            except Exception:
+                pass
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -203,7 +248,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "source": "nvml, 10 ms" if self.nvml is not None else "nvidia-smi, 100 ms"}
 
 
 # ----------------------------------------------------------------------------- our arm

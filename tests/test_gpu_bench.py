@@ -32,6 +32,10 @@ def test_bench_json_line_contract():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["gpu_launches"] == 5 * 4                        # fwd + 2 chunks + merge per step
     assert d["merge_roofline"]["bound"] == "hbm"
+    assert d["clocks"]["samples"] >= 1 and d["clocks"]["sm_mhz"] > 0
+    f = d["forwards"]
+    for key in ("sd3_1024_bf16", "flux_1024_bf16", "flux_2048_bf16", "video_bf16", "flux_2048_e4m3", "video_e4m3"):
+        assert f[key]["tflops"] > 0 and 0 < f[key]["frac"] < 2, (key, f[key])
 
 
 def test_bench_video_e2e_pipeline_matches():
