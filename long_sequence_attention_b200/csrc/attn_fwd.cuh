@@ -20,8 +20,8 @@
 //
 // Instantiations (template <D, FP8, NA, PARTS>): the dense form (bf16 D = 64 / 128, e4m3
 // D = 128, per-tensor or per-block scales, plain or sequence-segmented layouts, optional
-// running (O, LSE) accumulator); NA, 3-D neighborhood attention, where a tile is a 4x4x8
-// token brick and a unit visits only the KV bricks of its queries' windows, with per-row
+// running (O, LSE) accumulator); NA, 3-D neighborhood attention, where a tile is a brick of
+// tokens and each Q brick visits only the KV bricks of its own rows' windows, with per-row
 // window masks; PARTS, where the query and key rows lie in blocks held by several ranks
 // (possibly other GPUs) and every tile is loaded from the block that holds it.
 //
@@ -30,7 +30,8 @@
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    MMA issuer (one thread issues every tcgen05.mma and commit)
 //   warp  9    TMA producer (Q once, then a ring of K stages and a ring of V stages)
-//   warps 10-11 idle (they complete the third warpgroup)
+//   warp  10   NA only: TMA producer of Q tile 1's K and V tiles (warp 9 then loads tile 0's)
+//   warps 10-11 otherwise idle (they complete the third warpgroup)
 // The block launches with 168 registers per thread; the third warpgroup then gives
 // registers back (setmaxnreg.dec to kRegsCtl) and the softmax warpgroups take them
 // (setmaxnreg.inc to kRegsSoftmax): 2*128*216 + 128*72 = 64512 = 384*168, so the increase
@@ -81,10 +82,12 @@ struct AttnParams {
   // seg = S is the plain [B, H, S, D] layout.
   int seg_q, seg_kv;
   // Neighborhood attention (the NA instantiation only): T x Y x X token grid, odd window
-  // sizes, and the unit grid (Q bricks along t, brick pairs along y, bricks along x).
+  // sizes, the Q brick (t, y, x extents, product 128), the axis along which the two Q bricks
+  // of a unit lie next to each other (0 = t, 1 = y, 2 = x), and the unit grid.
   int na_T, na_Y, na_X;
   int na_Kt, na_Ky, na_Kx;
-  int na_nbt, na_nby2, na_nbx;
+  int na_qbt, na_qby, na_qbx, na_pax;
+  int na_nut, na_nuy, na_nux;
   // Parts (the PARTS instantiation only): the keys are n_kv_parts blocks and the queries
   // n_q_parts blocks of part_rows rows each, block p held by tensors [B, part_H, part_rows, D]
   // at (possibly a peer GPU's) addresses; this launch computes heads [part_h0, part_h0 + H)
@@ -110,21 +113,23 @@ struct MapSet {
 // section 5, reports it as the decoder's hot spot).  The neighborhood of a query at
 // position i along a dimension of length L is the K positions starting at
 // clamp(i - K/2, 0, L - K); the 3-D neighborhood is the product over (t, y, x).
-// A 128-row tile is a brick of kNaBt x kNaBy x kNaBx tokens, loaded by one 5-D TMA box
-// (x fastest), so tile row c is the token (c / 32, (c / 8) % 4, c % 8) of the brick.  A unit
-// is two bricks stacked along y; its KV tiles are bricks laid from the origin of the union of
-// its queries' windows (TMA boxes may start at any token; only the innermost D coordinate has
-// an alignment rule), and each row masks the keys outside its own window.
+// A 128-row Q tile is a brick of qbt x qby x qbx tokens and a KV tile a brick of
+// kNaBt x kNaBy x kNaBx tokens, each loaded by one 5-D TMA box (x fastest), so tile row c is
+// token (c / (by * bx), (c / bx) % by, c % bx) of its brick.  A unit is two Q bricks side by
+// side along one axis (the two ping-pong tiles); each Q brick has its own list of KV bricks,
+// laid from the origin of the union of its rows' windows (TMA boxes may start at any token;
+// only the innermost D coordinate has an alignment rule), and each row masks the keys outside
+// its own window.  A unit takes as many KV steps as the longer of its two lists; the other
+// tile's extra steps are empty (no exponentials, P = 0).
 // ---------------------------------------------------------------------------------------
 constexpr int kNaBt = 4, kNaBy = 4, kNaBx = 8;
 
 __device__ __forceinline__ int na_wstart(int i, int K, int L) { return min(max(i - K / 2, 0), L - K); }
 
-struct NaUnit {
-  int bh;
-  int qt, qy, qx;        // token origin of Q brick 0 (brick 1 is kNaBy further along y)
-  int ut, uy, ux;        // token origin of the union of the unit's windows
-  int nt, ny, nx;        // KV bricks along t, y, x
+struct NaTile {
+  int qt, qy, qx;        // token origin of the Q brick
+  int ut, uy, ux;        // token origin of the union of its rows' windows
+  int nt, ny, nx;        // KV bricks along t, y, x (all 0 for a Q brick past the grid)
   __device__ __forceinline__ int n() const { return nt * ny * nx; }
   // token origin of KV tile j (x fastest, then y, then t)
   __device__ __forceinline__ void kv_origin(int j, int& t, int& y, int& x) const {
@@ -136,26 +141,44 @@ struct NaUnit {
 };
 
 // Union [first, first + len) of the windows of the queries [a, min(a + ext, L)) along one
-// dimension (window starts never decrease with the position), covered by `count` bricks of b.
+// dimension (window starts never decrease with the position), covered by `count` bricks of b;
+// no queries (a >= L) gives count 0.
 __device__ __forceinline__ void na_span(int a, int ext, int K, int L, int b, int& first, int& count) {
+  if (a >= L) {
+    first = 0;
+    count = 0;
+    return;
+  }
   const int last = min(a + ext, L) - 1;
   first = na_wstart(a, K, L);
   count = (na_wstart(last, K, L) + K - first + b - 1) / b;
 }
 
-__device__ __forceinline__ NaUnit na_unit(const AttnParams& p, int u) {
-  NaUnit w;
-  const int per_bh = p.na_nbt * p.na_nby2 * p.na_nbx;
-  w.bh = u / per_bh;
-  const int r = u - w.bh * per_bh;
-  const int ix = r % p.na_nbx, iy = (r / p.na_nbx) % p.na_nby2, it = r / (p.na_nbx * p.na_nby2);
-  w.qt = it * kNaBt;
-  w.qy = iy * 2 * kNaBy;
-  w.qx = ix * kNaBx;
-  na_span(w.qt, kNaBt, p.na_Kt, p.na_T, kNaBt, w.ut, w.nt);
-  na_span(w.qy, 2 * kNaBy, p.na_Ky, p.na_Y, kNaBy, w.uy, w.ny);
-  na_span(w.qx, kNaBx, p.na_Kx, p.na_X, kNaBx, w.ux, w.nx);
+// Head index of unit u and Q tile t (0 or 1) of it.
+__device__ __forceinline__ int na_unit_bh(const AttnParams& p, int u) {
+  return u / (p.na_nut * p.na_nuy * p.na_nux);
+}
+__device__ __forceinline__ NaTile na_tile(const AttnParams& p, int u, int t) {
+  NaTile w;
+  const int per_bh = p.na_nut * p.na_nuy * p.na_nux;
+  const int r = u % per_bh;
+  const int ix = r % p.na_nux, iy = (r / p.na_nux) % p.na_nuy, it = r / (p.na_nux * p.na_nuy);
+  const int et = p.na_qbt * (p.na_pax == 0 ? 2 : 1);
+  const int ey = p.na_qby * (p.na_pax == 1 ? 2 : 1);
+  const int ex = p.na_qbx * (p.na_pax == 2 ? 2 : 1);
+  w.qt = it * et + (p.na_pax == 0 ? t * p.na_qbt : 0);
+  w.qy = iy * ey + (p.na_pax == 1 ? t * p.na_qby : 0);
+  w.qx = ix * ex + (p.na_pax == 2 ? t * p.na_qbx : 0);
+  na_span(w.qt, p.na_qbt, p.na_Kt, p.na_T, kNaBt, w.ut, w.nt);
+  na_span(w.qy, p.na_qby, p.na_Ky, p.na_Y, kNaBy, w.uy, w.ny);
+  na_span(w.qx, p.na_qbx, p.na_Kx, p.na_X, kNaBx, w.ux, w.nx);
+  if (w.nt == 0 || w.ny == 0 || w.nx == 0) w.nt = w.ny = w.nx = 0;
   return w;
+}
+
+// KV steps of unit u: the longer of its two tiles' lists (tile 0 always lies in the grid).
+__device__ __forceinline__ int na_steps(const AttnParams& p, int u) {
+  return max(na_tile(p, u, 0).n(), na_tile(p, u, 1).n());
 }
 
 // 128-bit key mask of one query row for a KV brick at token origin (ot, oy, ox): bit c set
@@ -375,8 +398,9 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     regs_dec<C::kRegsCtl>();
-  if (warp == C::kTmaWarp) {
+  if (warp == C::kTmaWarp || (NA && warp == C::kTmaWarp + 1)) {
     // ------------------------------------------------------------------ TMA producer
+    // (NA: warp 9 loads Q and the K / V tiles of Q tile 0, warp 10 those of Q tile 1)
     if (lane == 0) {
       if constexpr (PARTS) {
         for (int pt = 0; pt < p.n_q_parts; ++pt) tma_prefetch_desc(&maps.q[pt]);
@@ -390,26 +414,63 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tm_v);
       }
       int k_issued = 0, v_issued = 0, q_issued = 0;   // running counts over all units
-      int g0 = 0;                                      // running KV tile count at unit start
       bool ok = true;
-      for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
-        NaUnit w;
-        int bh, q0, nkv;
-        if constexpr (NA) {
-          w = na_unit(p, u);
-          bh = w.bh; q0 = 0; nkv = w.n();
-        } else {
-          bh = unit_bh(u); q0 = unit_q0(u); nkv = n_kv;
+      const int lt = warp - C::kTmaWarp;               // NA: the Q tile whose K / V this thread loads
+      if constexpr (NA) {
+        // Each Q tile has its own ring of K slots (lt, lt + 2, ...) and of V slots; K(j + 1)
+        // reuses the slot of K(j + 1 - kKPer), freed when that tile's S MMA is done, and
+        // V(j + 1) the slot freed by its P.V.
+        constexpr int kKPer = C::kKStages / 2, kVPer = C::kVStages / 2;
+        int G = 0;                                     // running KV step count at unit start
+        for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+          const int bh = na_unit_bh(p, u);
+          const NaTile w0 = na_tile(p, u, 0), w1 = na_tile(p, u, 1);
+          const int n = max(w0.n(), w1.n());
+          if (lt == 0) {
+            // Q of this unit may overwrite the previous unit's only after its last S MMA.
+            if (it > 0 && !(ok = mbar_wait(bar_q_empty, (it - 1) & 1, abort_flag, tmo, 0))) break;
+            mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
+            for (int b = 0; b < C::kNBlk; ++b) {
+              tma_load_5d(sQ + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner, w0.qx, w0.qy, w0.qt, bh);
+              tma_load_5d(sQ + C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner, w1.qx, w1.qy,
+                          w1.qt, bh);
+            }
+            q_issued = it + 1;
+          }
+          // a step past the tile's own list (its P is 0) reloads one of its bricks (or, for a
+          // Q brick past the grid, one of tile 0's) so that the MMA reads finite data
+          const NaTile& w = (lt ? w1 : w0).n() > 0 ? (lt ? w1 : w0) : w0;
+          for (int j = 0; j < n; ++j) {
+            int ot, oy, ox;
+            w.kv_origin(min(j, w.n() - 1), ot, oy, ox);
+            const int i = G + j;
+            const int ks = lt + 2 * (i % kKPer);
+            if (i >= kKPer && !(ok = mbar_wait(bar_k_empty + ks, ((i / kKPer) + 1) & 1, abort_flag, tmo, 1))) break;
+            mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
+            for (int b = 0; b < C::kNBlk; ++b)
+              tma_load_5d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks, b * C::kBoxInner, ox,
+                          oy, ot, bh);
+            k_issued = i + 1;
+            const int vs = lt + 2 * (i % kVPer);
+            if (i >= kVPer && !(ok = mbar_wait(bar_v_empty + vs, ((i / kVPer) + 1) & 1, abort_flag, tmo, 2))) break;
+            mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
+            for (int b = 0; b < C::kNBlk; ++b)
+              tma_load_5d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs, b * C::kBoxInner, ox,
+                          oy, ot, bh);
+            v_issued = i + 1;
+          }
+          G += n;
         }
+      } else {
+      int g0 = 0;                                      // running KV tile count at unit start
+      for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+        const int bh = unit_bh(u), q0 = unit_q0(u), nkv = n_kv;
         // Q of this unit may overwrite the previous unit's only after its last S MMA.
         if (it > 0 && !(ok = mbar_wait(bar_q_empty, (it - 1) & 1, abort_flag, tmo, 0))) break;
         mbar_arrive_expect_tx(bar_q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int b = 0; b < C::kNBlk; ++b) {
-            if constexpr (NA)
-              tma_load_5d(sQ + t * C::kTileBytes + b * C::kBlkBytes, &tm_q, bar_q_full, b * C::kBoxInner, w.qx,
-                          w.qy + t * kNaBy, w.qt, bh);
-            else if constexpr (PARTS) {
+            if constexpr (PARTS) {
               // row -> (part, row in part); rows past the last part read as zero (past its end)
               const int row = q0 + t * C::kBM;
               const int pt = min(row / p.part_rows, p.n_q_parts - 1);
@@ -423,18 +484,13 @@ __global__ void __launch_bounds__(384, 1)
         for (int j = 0; j < nkv; ++j) {
           const int g = g0 + j;
           const int kv_row = p.k0 + j * C::kBN;
-          int ot = 0, oy = 0, ox = 0;
-          if constexpr (NA) w.kv_origin(j, ot, oy, ox);
           const int ks = g % C::kKStages;
           if (g >= C::kKStages &&
               !(ok = mbar_wait(bar_k_empty + ks, ((g / C::kKStages) + 1) & 1, abort_flag, tmo, 1)))
             break;
           mbar_arrive_expect_tx(bar_k_full + ks, C::kTileBytes);
           for (int b = 0; b < C::kNBlk; ++b) {
-            if constexpr (NA)
-              tma_load_5d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &tm_k, bar_k_full + ks, b * C::kBoxInner,
-                          ox, oy, ot, bh);
-            else if constexpr (PARTS) {
+            if constexpr (PARTS) {
               const int pt = min(kv_row / p.part_rows, p.n_kv_parts - 1);
               tma_load_4d(sK + ks * C::kTileBytes + b * C::kBlkBytes, &maps.k[pt], bar_k_full + ks,
                           b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
@@ -449,10 +505,7 @@ __global__ void __launch_bounds__(384, 1)
             break;
           mbar_arrive_expect_tx(bar_v_full + vs, C::kTileBytes);
           for (int b = 0; b < C::kNBlk; ++b) {
-            if constexpr (NA)
-              tma_load_5d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &tm_v, bar_v_full + vs, b * C::kBoxInner,
-                          ox, oy, ot, bh);
-            else if constexpr (PARTS) {
+            if constexpr (PARTS) {
               const int pt = min(kv_row / p.part_rows, p.n_kv_parts - 1);
               tma_load_4d(sV + vs * C::kTileBytes + b * C::kBlkBytes, &maps.v[pt], bar_v_full + vs,
                           b * C::kBoxInner, kv_row - pt * p.part_rows, bh % p.H, bh / p.H);
@@ -464,16 +517,20 @@ __global__ void __launch_bounds__(384, 1)
         }
         g0 += nkv;
       }
+      }
       // Drain: the last load armed on every stage must land before the CTA may exit
       // (a no-op in a healthy run, where the consumers already waited for all of them).
+      // (NA: this thread's ring is the slots lt + 2 r, with per-tile counts)
+      constexpr int kKRing = NA ? C::kKStages / 2 : C::kKStages, kVRing = NA ? C::kVStages / 2 : C::kVStages;
+      const int slot_step = NA ? 2 : 1, slot0 = NA ? lt : 0;
       if (q_issued > 0) mbar_wait_drain(bar_q_full, (q_issued - 1) & 1, tmo);
-      for (int s = 0; s < C::kKStages; ++s) {
-        const int last = s + ((k_issued - 1 - s) / C::kKStages) * C::kKStages;
-        if (k_issued > s) mbar_wait_drain(bar_k_full + s, (last / C::kKStages) & 1, tmo);
+      for (int r = 0; r < kKRing; ++r) {
+        const int last = r + ((k_issued - 1 - r) / kKRing) * kKRing;
+        if (k_issued > r) mbar_wait_drain(bar_k_full + slot0 + slot_step * r, (last / kKRing) & 1, tmo);
       }
-      for (int s = 0; s < C::kVStages; ++s) {
-        const int last = s + ((v_issued - 1 - s) / C::kVStages) * C::kVStages;
-        if (v_issued > s) mbar_wait_drain(bar_v_full + s, (last / C::kVStages) & 1, tmo);
+      for (int r = 0; r < kVRing; ++r) {
+        const int last = r + ((v_issued - 1 - r) / kVRing) * kVRing;
+        if (v_issued > r) mbar_wait_drain(bar_v_full + slot0 + slot_step * r, (last / kVRing) & 1, tmo);
       }
     }
   } else if (warp == C::kMmaWarp) {
@@ -517,11 +574,67 @@ __global__ void __launch_bounds__(384, 1)
       };
 
       bool ok = true;
+      if constexpr (NA) {
+        // The two Q tiles have their own K and V tiles and their own ring slots (tile t uses
+        // slots t, t + 2, ...), so they are independent pipelines: this thread issues a
+        // tile's next P.V + S as soon as that tile's P and K / V tiles are ready, in whatever
+        // order the two tiles get there, and never holds one tile back behind the other.
+        constexpr int kKPer = C::kKStages / 2, kVPer = C::kVStages / 2;
+        int G = 0;                                     // running KV step count at unit start
+        PollGuard guard;
+        // steps of the next unit, computed while this thread waits anyway (at a unit boundary
+        // the softmax warpgroups' epilogue stores make every instruction here slow)
+        int n_next = blockIdx.x < p.n_units ? na_steps(p, blockIdx.x) : 0;
+        for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
+          const int n = n_next;
+          if (!(ok = mbar_wait(bar_q_full, it & 1, abort_flag, tmo, 3))) break;
+          n_next = u + static_cast<int>(gridDim.x) < p.n_units ? na_steps(p, u + gridDim.x) : 0;
+          tc_fence_after();
+          // js[t] = j: the tile's next action issues P.V(j - 1) (j > 0) and S(j) (j < n)
+          int js[2] = {0, 0};
+          bool q_released = false;
+          while (ok && (js[0] <= n || js[1] <= n)) {
+            bool progress = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              const int j = js[t];
+              if (j > n) continue;
+              const int ik = G + j, iv = G + j - 1;
+              const int ks = t + 2 * (ik % kKPer), vs = t + 2 * ((iv + kVPer) % kVPer);
+              if (j < n && !mbar_test(bar_k_full + ks, (ik / kKPer) & 1)) continue;
+              if (j > 0 && !(mbar_test(bar_v_full + vs, (iv / kVPer) & 1) && mbar_test(bar_p_full + t, iv & 1)))
+                continue;
+              tc_fence_after();
+              if (j > 0) {
+                issue_pv(t, vs, j > 1);
+                if (j == n) tc_commit(bar_o_final + t);
+                tc_commit(bar_v_empty + vs);
+              }
+              if (j < n) {
+                issue_s(t, ks);
+                tc_commit(bar_s_full + t);
+                tc_commit(bar_k_empty + ks);
+              }
+              js[t] = j + 1;
+              progress = true;
+            }
+            if (!q_released && js[0] >= n && js[1] >= n) {
+              tc_commit(bar_q_empty);                  // every S MMA of this unit is issued
+              q_released = true;
+            }
+            if (progress) {
+              guard.progress();
+            } else {
+              ok = guard.idle(abort_flag, tmo, 4);
+              __nanosleep(20);                         // leave the issue slots to the softmax warps
+            }
+          }
+          G += n;
+        }
+      } else {
       int g0 = 0;                                      // running KV tile count at unit start
       for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
-        int nkv;
-        if constexpr (NA) nkv = na_unit(p, u).n();
-        else nkv = n_kv;
+        const int nkv = n_kv;
         if (!(ok = mbar_wait(bar_q_full, it & 1, abort_flag, tmo, 3))) break;
         tc_fence_after();
         for (int j = 0; ok && j < nkv; ++j) {
@@ -567,11 +680,12 @@ __global__ void __launch_bounds__(384, 1)
         }
         g0 += nkv;
       }
+      }
       // Every MMA this thread issued must finish before TMEM is released.
       tc_commit(bar_drain);
       mbar_wait_drain(bar_drain, 0, tmo);
     }
-  }  // warps 10 and 11 have no role
+  }  // warp 11 (and warp 10 outside NA) has no role
   } else {
     // ------------------------------------------------------------------ softmax warpgroups
     regs_inc<C::kRegsSoftmax>();
@@ -601,15 +715,16 @@ __global__ void __launch_bounds__(384, 1)
 
     int g0 = 0;                                                // running KV tile count at unit start
     for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
-    NaUnit w;
-    int bh, q_start, nkv;
+    NaTile w;
+    int bh, q_start, nkv, n_own = 0;     // NA: n_own = KV bricks of this tile's own list
     int qt = 0, qy = 0, qx = 0, wt = 0, wy = 0, wx = 0;       // NA: this row's token and window starts
     if constexpr (NA) {
-      w = na_unit(p, u);
-      bh = w.bh; q_start = 0; nkv = w.n();
-      qt = w.qt + row / (kNaBy * kNaBx);
-      qy = w.qy + t * kNaBy + (row / kNaBx) % kNaBy;
-      qx = w.qx + row % kNaBx;
+      w = na_tile(p, u, t);
+      n_own = w.n();
+      bh = na_unit_bh(p, u); q_start = 0; nkv = max(n_own, na_tile(p, u, t ^ 1).n());
+      qt = w.qt + row / (p.na_qby * p.na_qbx);
+      qy = w.qy + (row / p.na_qbx) % p.na_qby;
+      qx = w.qx + row % p.na_qbx;
       wt = na_wstart(qt, p.na_Kt, p.na_T);
       wy = na_wstart(qy, p.na_Ky, p.na_Y);
       wx = na_wstart(qx, p.na_Kx, p.na_X);
@@ -655,6 +770,15 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar_s_full + t, g & 1, abort_flag, tmo, 11 + t));
       if (!ok) break;
       tc_fence_after();
+      uint32_t pw[2 * C::kPWordsHalf];
+      float sum = 0.0f;
+      float alpha = 1.0f;
+      bool need = false;
+      if (NA && j >= n_own) {
+        // a step past this tile's own KV list (the other tile's list is longer): no keys, P = 0
+#pragma unroll
+        for (int i = 0; i < 2 * C::kPWordsHalf; ++i) pw[i] = 0u;
+      } else {
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
       const int valid = p.k1 - (p.k0 + j * C::kBN);
@@ -674,10 +798,6 @@ __global__ void __launch_bounds__(384, 1)
       // kSumBound), the usual case after the first tile.  Otherwise (first tile, a row max
       // that rose a lot, or the e4m3 path) the warp takes the exact route: (re)load S (still
       // intact in TMEM, P is not written yet), exact row max, rescale, exponentiate.
-      uint32_t pw[2 * C::kPWordsHalf];
-      float sum;
-      float alpha = 1.0f;
-      bool need = false;
       // (NA: a row whose window has missed every tile so far has no max yet: exact route)
       bool slow = (j == 0) || !C::kSpeculative || (NA && __any_sync(0xffffffffu, m_use == -INFINITY));
       if (!slow) {
@@ -713,6 +833,7 @@ __global__ void __launch_bounds__(384, 1)
           const float mc = (NA && m_use == -INFINITY) ? 0.0f : m_use * cl;
           exp_pass<FP8, C::kEmuMask>(s, cl, mc - C::kPShift, pw, sum);
         }
+      }
       }
       tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pw[0]));
       if constexpr (!FP8) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pw[32]));

@@ -1,5 +1,6 @@
 // C-ABI boundary of the DiT attention library: argument validation, TMA descriptor
 // construction, kernel launches and status codes.  See include/dit_attn.h for the contract.
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -91,9 +92,9 @@ int make_map(CUtensorMap* m, const void* ptr, bool fp8, int D, int S, int BH, in
 }
 
 // 5-D map (D, X, Y, T, BH) of a bf16 [BH, T*Y*X, D] tensor on a T x Y x X token grid for
-// the neighborhood-attention kernel.  Box: 128 bytes x an 8 x 4 x 4 (x, y, t) brick of
-// tokens = 128 rows, 128-byte swizzle; tokens past the grid read as zero.
-int make_map_na(CUtensorMap* m, const void* ptr, int D, int T, int Y, int X, int BH) {
+// the neighborhood-attention kernel.  Box: 128 bytes x a bx x by x bt (x, y, t) brick of
+// tokens (bx * by * bt = 128 rows), 128-byte swizzle; tokens past the grid read as zero.
+int make_map_na(CUtensorMap* m, const void* ptr, int D, int T, int Y, int X, int BH, int bt, int by, int bx) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return DIT_ERR_CUDA;
   const cuuint64_t e = 2;
@@ -101,13 +102,71 @@ int make_map_na(CUtensorMap* m, const void* ptr, int D, int T, int Y, int X, int
                         static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[4] = {static_cast<cuuint64_t>(D) * e, static_cast<cuuint64_t>(X) * D * e,
                            static_cast<cuuint64_t>(Y) * X * D * e, static_cast<cuuint64_t>(T) * Y * X * D * e};
-  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / e), static_cast<cuuint32_t>(kNaBx),
-                       static_cast<cuuint32_t>(kNaBy), static_cast<cuuint32_t>(kNaBt), 1};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / e), static_cast<cuuint32_t>(bx), static_cast<cuuint32_t>(by),
+                       static_cast<cuuint32_t>(bt), 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? DIT_OK : DIT_ERR_CUDA;
+}
+
+// Q brick and pairing axis of the neighborhood kernel for a grid and window.  Each Q brick
+// (t, y, x extents, powers of two with product 128) visits the KV bricks that cover the union
+// of its rows' windows, and a unit (two Q bricks side by side along axis pax) takes as many
+// KV steps as the longer of its two lists.  The choice minimises the steps of a head plus
+// kNaUnitCost steps for every unit (the epilogue and the next Q load of a unit boundary).
+// The step count factorises over the dimensions: a brick's list length is the product of
+// its per-dimension brick counts, and the two bricks of a unit differ along pax only.
+constexpr long long kNaUnitCost = 2;
+
+int na_host_wstart(int i, int K, int L) { return std::min(std::max(i - K / 2, 0), L - K); }
+
+// KV bricks of extent b covering the windows of the queries [a, min(a + ext, L)); 0 if a >= L.
+long long na_host_count(int a, int ext, int K, int L, int b) {
+  if (a >= L) return 0;
+  const int last = std::min(a + ext, L) - 1;
+  const int first = na_host_wstart(a, K, L);
+  return (na_host_wstart(last, K, L) + K - first + b - 1) / b;
+}
+
+struct NaChoice {
+  int qb[3];   // Q brick extents (t, y, x)
+  int pax;     // axis of the unit's brick pair
+  int nu[3];   // units along t, y, x
+};
+
+NaChoice na_choose(const int L[3], const int K[3]) {
+  static const int kb[3] = {kNaBt, kNaBy, kNaBx};
+  NaChoice best{{kNaBt, kNaBy, kNaBx}, 1, {0, 0, 0}};
+  long long best_cost = -1;
+  for (int lt = 0; lt <= 7; ++lt)
+    for (int ly = 0; lt + ly <= 7; ++ly) {
+      const int qb[3] = {1 << lt, 1 << ly, 1 << (7 - lt - ly)};
+      for (int pax = 0; pax < 3; ++pax) {
+        long long steps = 1, units = 1;
+        int nu[3];
+        for (int d = 0; d < 3; ++d) {
+          const int e = qb[d] * (d == pax ? 2 : 1);
+          nu[d] = (L[d] + e - 1) / e;
+          long long sd = 0;
+          for (int i = 0; i < nu[d]; ++i) {
+            const int o = i * e;
+            long long c = na_host_count(o, qb[d], K[d], L[d], kb[d]);
+            if (d == pax) c = std::max(c, na_host_count(o + qb[d], qb[d], K[d], L[d], kb[d]));
+            sd += c;
+          }
+          steps *= sd;
+          units *= nu[d];
+        }
+        const long long cost = steps + kNaUnitCost * units;
+        if (best_cost < 0 || cost < best_cost) {
+          best_cost = cost;
+          best = NaChoice{{qb[0], qb[1], qb[2]}, pax, {nu[0], nu[1], nu[2]}};
+        }
+      }
+    }
+  return best;
 }
 
 // Number of SMs of the current device (cached per device).
@@ -217,13 +276,15 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
     if (units > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
     pr.n_units = static_cast<int>(units);
   } else if constexpr (NA) {
-    if ((rc = make_map_na(&tq, q, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
-    if ((rc = make_map_na(&tk, k, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
-    if ((rc = make_map_na(&tv, v, D, prm.na_T, prm.na_Y, prm.na_X, BH)) != DIT_OK) return rc;
-    pr.na_nbt = (prm.na_T + kNaBt - 1) / kNaBt;
-    pr.na_nby2 = (prm.na_Y + 2 * kNaBy - 1) / (2 * kNaBy);
-    pr.na_nbx = (prm.na_X + kNaBx - 1) / kNaBx;
-    const long long units = static_cast<long long>(BH) * pr.na_nbt * pr.na_nby2 * pr.na_nbx;
+    const int L[3] = {prm.na_T, prm.na_Y, prm.na_X}, K[3] = {prm.na_Kt, prm.na_Ky, prm.na_Kx};
+    const NaChoice ch = na_choose(L, K);
+    if ((rc = make_map_na(&tq, q, D, prm.na_T, prm.na_Y, prm.na_X, BH, ch.qb[0], ch.qb[1], ch.qb[2])) != DIT_OK)
+      return rc;
+    if ((rc = make_map_na(&tk, k, D, prm.na_T, prm.na_Y, prm.na_X, BH, kNaBt, kNaBy, kNaBx)) != DIT_OK) return rc;
+    if ((rc = make_map_na(&tv, v, D, prm.na_T, prm.na_Y, prm.na_X, BH, kNaBt, kNaBy, kNaBx)) != DIT_OK) return rc;
+    pr.na_qbt = ch.qb[0]; pr.na_qby = ch.qb[1]; pr.na_qbx = ch.qb[2]; pr.na_pax = ch.pax;
+    pr.na_nut = ch.nu[0]; pr.na_nuy = ch.nu[1]; pr.na_nux = ch.nu[2];
+    const long long units = static_cast<long long>(BH) * ch.nu[0] * ch.nu[1] * ch.nu[2];
     if (units > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
     pr.n_qblk = 0;
     pr.n_units = static_cast<int>(units);

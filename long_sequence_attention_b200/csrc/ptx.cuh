@@ -65,6 +65,40 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return ok != 0;
 }
 
+// Non-blocking test: has the phase of the barrier with the given parity completed?
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bookkeeping of a polling loop that tests several barriers without blocking: call idle()
+// on every pass that made no progress.  It gives up like mbar_wait (abort flag, or
+// timeout_ns of wall time without progress, recorded with `site`) and returns false then.
+struct PollGuard {
+  uint64_t t0 = 0;
+  uint32_t it = 0;
+  __device__ __forceinline__ void progress() { it = 0; }
+  __device__ __forceinline__ bool idle(volatile int* abort_flag, uint64_t timeout_ns, uint32_t site) {
+    if (it == 0) t0 = global_timer_ns();
+    ++it;
+    if ((it & 63u) != 0u) return true;
+    if (*abort_flag) return false;
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicOr(&g_error_word, kErrTimeout | (site << 8));
+      *abort_flag = 1;
+      return false;
+    }
+    return true;
+  }
+};
+
 // Wait for the phase of `bar` with the given parity to complete.  Never spins forever:
 // gives up when the CTA's `abort_flag` (shared memory) is set, or after `timeout_ns` of
 // wall time; on a timeout it records kErrTimeout | (site << 8) in the device error word and
