@@ -137,8 +137,11 @@ int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, flo
  *
  *   q, k, v   [B,H,T*Y*X,D] bf16;  out [B,H,T*Y*X,D] bf16;  lse [B,H,T*Y*X] fp32 or NULL.
  *   Kt, Ky, Kx odd, 1 <= K <= the grid dimension, else DIT_ERR_INVALID_ARG.  D = 64 or 128.
- *   The kernel visits only the 128-token bricks (4 x 4 x 8 in t, y, x) that some window of
- *   its queries touches and masks, per query, the keys outside that query's window.
+ *   scale >= 1e-20 (else DIT_ERR_INVALID_ARG); scores |q . k| below 1e27.
+ *   Each 128-query brick of the grid (its shape chosen per call from the grid and window)
+ *   visits only the 128-key bricks (4 x 4 x 8 in t, y, x) that cover its queries' windows; the
+ *   keys of a brick outside a query's window get a score penalty of -2^100 (an extra step of
+ *   the score MMA), so their weights are exactly 0.
  */
 int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
                  int T, int Y, int X, int D, int Kt, int Ky, int Kx, float scale, void* stream);

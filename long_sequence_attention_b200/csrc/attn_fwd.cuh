@@ -181,27 +181,61 @@ __device__ __forceinline__ int na_steps(const AttnParams& p, int u) {
   return max(na_tile(p, u, 0).n(), na_tile(p, u, 1).n());
 }
 
-// 128-bit key mask of one query row for a KV brick at token origin (ot, oy, ox): bit c set
-// when key c of the brick lies in the row's window [ws, ws + K) along every dimension.
-// Word w covers brick plane t = w (4 y-rows of 8 x-bits).
-__device__ __forceinline__ void na_row_mask(int wt, int wy, int wx, int Kt, int Ky, int Kx, int ot, int oy, int ox,
-                                            uint32_t (&mw)[4]) {
-  const int lx = min(max(wx - ox, 0), kNaBx), hx = min(max(wx + Kx - ox, 0), kNaBx);
-  const int ly = min(max(wy - oy, 0), kNaBy), hy = min(max(wy + Ky - oy, 0), kNaBy);
-  const int lt = wt - ot, ht = wt + Kt - ot;
-  const uint32_t xbits = ((1u << hx) - 1u) & ~((1u << lx) - 1u);          // <= 8 bits
-  uint32_t ymul = 0u;
+// Window penalties.  Every S tile of the NA form gets one more K = 16 MMA step: a 16-feature
+// row per query (A operand) times a 16-feature row per key (B operand).  Key c of a KV brick
+// carries one-hot features of its brick position: feature ct = c / 32 (t), 4 + cy with
+// cy = (c / 8) % 4 (y), 8 + cx with cx = c % 8 (x).  A query row carries, for the brick being
+// visited, -kNaPen at each position whose coordinate lies outside its window along that axis
+// and 0 elsewhere, so the extra step adds 0 to every key in the row's window (exact) and at
+// most -3 kNaPen to the others, whose exponentials then vanish.  Both operands are K-major
+// without swizzle: row r's 32 bytes at (r / 8) * 256 + (r % 8) * 16, features 8-15 128 bytes
+// further on.
+constexpr uint32_t kNaPenBits = 0xF180u;   // bf16 -2^100
+constexpr uint32_t kNaOneBits = 0x3F80u;   // bf16 1.0
+constexpr int kNaXBytes = 128 * 32;        // one 128-row feature block
+
+// Write the penalty features of one query row (window starts wt, wy, wx) for the KV brick at
+// token origin (ot, oy, ox) into block sX.
+__device__ __forceinline__ void na_write_pen(uint8_t* sX, int row, int wt, int wy, int wx, int Kt, int Ky, int Kx,
+                                             int ot, int oy, int ox) {
+  auto pen = [](int v, int lo, int K) -> uint32_t { return (v >= lo && v < lo + K) ? 0u : kNaPenBits; };
+  uint32_t h[8];
 #pragma unroll
-  for (int cy = 0; cy < kNaBy; ++cy) ymul |= (cy >= ly && cy < hy) ? (1u << (8 * cy)) : 0u;
-  const uint32_t plane = xbits * ymul;                                     // no carries: xbits < 256
+  for (int i = 0; i < 2; ++i) {
+    h[i] = pen(ot + 2 * i, wt, Kt) | (pen(ot + 2 * i + 1, wt, Kt) << 16);
+    h[2 + i] = pen(oy + 2 * i, wy, Ky) | (pen(oy + 2 * i + 1, wy, Ky) << 16);
+  }
 #pragma unroll
-  for (int ct = 0; ct < kNaBt; ++ct) mw[ct] = (ct >= lt && ct < ht) ? plane : 0u;
+  for (int i = 0; i < 4; ++i) h[4 + i] = pen(ox + 2 * i, wx, Kx) | (pen(ox + 2 * i + 1, wx, Kx) << 16);
+  uint8_t* base = sX + (row >> 3) * 256 + (row & 7) * 16;
+  *reinterpret_cast<uint4*>(base) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(base + 128) = make_uint4(h[4], h[5], h[6], h[7]);
 }
 
-__device__ __forceinline__ void apply_mask128(uint32_t (&s)[128], const uint32_t (&mw)[4]) {
+// Write the one-hot position features of key c of a KV brick into block sX.
+__device__ __forceinline__ void na_write_keyfeat(uint8_t* sX, int c) {
+  const int ft = c >> 5, fy = 4 + ((c >> 3) & 3), fx = 8 + (c & 7);
+  uint32_t h[8];
 #pragma unroll
-  for (int c = 0; c < 128; ++c)
-    if (!((mw[c >> 5] >> (c & 31)) & 1u)) s[c] = 0xFF800000u;
+  for (int i = 0; i < 8; ++i) {
+    const int f0 = 2 * i, f1 = 2 * i + 1;
+    h[i] = ((f0 == ft || f0 == fy || f0 == fx) ? kNaOneBits : 0u) |
+           (((f1 == ft || f1 == fy || f1 == fx) ? kNaOneBits : 0u) << 16);
+  }
+  uint8_t* base = sX + (c >> 3) * 256 + (c & 7) * 16;
+  *reinterpret_cast<uint4*>(base) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(base + 128) = make_uint4(h[4], h[5], h[6], h[7]);
+}
+
+// Token of row `row` of Q brick w and the starts of its window.
+__device__ __forceinline__ void na_row_geo(const AttnParams& p, const NaTile& w, int row, int& qt, int& qy, int& qx,
+                                           int& wt, int& wy, int& wx) {
+  qt = w.qt + row / (p.na_qby * p.na_qbx);
+  qy = w.qy + (row / p.na_qbx) % p.na_qby;
+  qx = w.qx + row % p.na_qbx;
+  wt = na_wstart(qt, p.na_Kt, p.na_T);
+  wy = na_wstart(qy, p.na_Ky, p.na_Y);
+  wx = na_wstart(qx, p.na_Kx, p.na_X);
 }
 
 // exp2 on the FMA pipe, two values at once with packed fp32x2 instructions: x = n + f with
@@ -272,12 +306,22 @@ struct AttnCfg {
   static constexpr int kOffK = kOffQ + 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kVStages * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1 + 2;
   static constexpr int kOffMisc = kOffBar + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(!FP8 || D == 128, "e4m3 path is built for D = 128");
+};
+
+// Shared memory of one launch.  The NA form adds the window-penalty features after the
+// barriers: one 4 KB block per Q tile and one for the keys.
+template <int D, bool FP8, bool NA>
+struct AttnSmem {
+  using C = AttnCfg<D, FP8>;
+  static constexpr int kOffX = ((C::kOffMisc + 16 + 1023) / 1024) * 1024;
+  static constexpr int kBytes = NA ? kOffX + 3 * kNaXBytes + 1024 : C::kSmemBytes;
+  static_assert(kBytes <= 227 * 1024, "shared memory budget");
 };
 
 // Columns c >= valid of a 128-column score row become -inf (keys past the range).
@@ -358,6 +402,7 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* bar_o_final = bar_p_full + 2;             // [2]
   uint64_t* bar_drain = bar_o_final + 2;              // [1]
   uint64_t* bar_q_empty = bar_drain + 1;              // [1]
+  uint64_t* bar_x0 = bar_q_empty + 1;                 // [2] NA: first penalty features written
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -380,6 +425,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar_drain, 1);
     mbar_init(bar_q_empty, 1);
+    mbar_init(bar_x0, 4);
+    mbar_init(bar_x0 + 1, 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -549,6 +596,10 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t qk_hi = static_cast<uint32_t>(dq >> 32), v_hi = static_cast<uint32_t>(dv >> 32);
       const uint32_t q_lo = static_cast<uint32_t>(dq), k_lo = static_cast<uint32_t>(dk),
                      v_lo = static_cast<uint32_t>(dv);
+      // NA: window-penalty features (query rows of tile t, keys), no swizzle, K-major
+      uint8_t* sX = smem + AttnSmem<D, FP8, NA>::kOffX;
+      const uint64_t dx = smem_desc_noswz(smem_u32(sX), 128, 256);
+      const uint32_t x_lo = static_cast<uint32_t>(dx), x_hi = static_cast<uint32_t>(dx >> 32);
       auto issue_s = [&](int t, int ks) {
         const uint32_t a0 = q_lo + ((t * C::kTileBytes) >> 4);
         const uint32_t b0 = k_lo + ((ks * C::kTileBytes) >> 4);
@@ -558,6 +609,8 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t off = ((kk * 32 / 128) * C::kBlkBytes + (kk * 32) % 128) >> 4;
           mma_ss_lohi(FP8, d, a0 + off, qk_hi, b0 + off, qk_hi, id_s, kk > 0 ? 1u : 0u);
         }
+        if constexpr (NA)
+          mma_ss_lohi(false, d, x_lo + ((t * kNaXBytes) >> 4), x_hi, x_lo + ((2 * kNaXBytes) >> 4), x_hi, id_s, 1u);
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
         const uint32_t b0 = v_lo + ((vs * C::kTileBytes) >> 4);
@@ -585,6 +638,10 @@ __global__ void __launch_bounds__(384, 1)
         // steps of the next unit, computed while this thread waits anyway (at a unit boundary
         // the softmax warpgroups' epilogue stores make every instruction here slow)
         int n_next = blockIdx.x < p.n_units ? na_steps(p, blockIdx.x) : 0;
+        // the softmax warpgroups have written the key features and each tile's first
+        // penalty features (later ones are written before the P that precedes their S)
+        if (blockIdx.x < p.n_units)
+          ok = mbar_wait(bar_x0, 0, abort_flag, tmo, 3) && mbar_wait(bar_x0 + 1, 0, abort_flag, tmo, 3);
         for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
           const int n = n_next;
           if (!(ok = mbar_wait(bar_q_full, it & 1, abort_flag, tmo, 3))) break;
@@ -714,6 +771,23 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
 
     int g0 = 0;                                                // running KV tile count at unit start
+    uint8_t* sX = smem + AttnSmem<D, FP8, NA>::kOffX;          // NA: window-penalty features
+    if constexpr (NA) {
+      // the keys' position features (static), and each tile's features for its first step
+      if (blockIdx.x < p.n_units) {
+        if (t == 0) na_write_keyfeat(sX + 2 * kNaXBytes, row);
+        const NaTile w0 = na_tile(p, blockIdx.x, t);
+        if (w0.n() > 0) {
+          int a, b, c, wt0, wy0, wx0, ot, oy, ox;
+          na_row_geo(p, w0, row, a, b, c, wt0, wy0, wx0);
+          w0.kv_origin(0, ot, oy, ox);
+          na_write_pen(sX + t * kNaXBytes, row, wt0, wy0, wx0, p.na_Kt, p.na_Ky, p.na_Kx, ot, oy, ox);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_x0 + t);
+      }
+    }
     for (int it = 0, u = blockIdx.x; ok && u < p.n_units; ++it, u += gridDim.x) {
     NaTile w;
     int bh, q_start, nkv, n_own = 0;     // NA: n_own = KV bricks of this tile's own list
@@ -722,12 +796,7 @@ __global__ void __launch_bounds__(384, 1)
       w = na_tile(p, u, t);
       n_own = w.n();
       bh = na_unit_bh(p, u); q_start = 0; nkv = max(n_own, na_tile(p, u, t ^ 1).n());
-      qt = w.qt + row / (p.na_qby * p.na_qbx);
-      qy = w.qy + (row / p.na_qbx) % p.na_qby;
-      qx = w.qx + row % p.na_qbx;
-      wt = na_wstart(qt, p.na_Kt, p.na_T);
-      wy = na_wstart(qy, p.na_Ky, p.na_Y);
-      wx = na_wstart(qx, p.na_Kx, p.na_X);
+      na_row_geo(p, w, row, qt, qy, qx, wt, wy, wx);
     } else {
       bh = unit_bh(u); q_start = unit_q0(u); nkv = n_kv;
     }
@@ -782,15 +851,8 @@ __global__ void __launch_bounds__(384, 1)
       uint32_t s[128];
       tmem_ld128_sync(tS, s);
       const int valid = p.k1 - (p.k0 + j * C::kBN);
-      uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};
-      bool part = false;                   // NA: some key of this tile lies outside the row's window
-      if constexpr (NA) {
-        int ot, oy, ox;
-        w.kv_origin(j, ot, oy, ox);
-        na_row_mask(wt, wy, wx, p.na_Kt, p.na_Ky, p.na_Kx, ot, oy, ox, mw);
-        part = (mw[0] & mw[1] & mw[2] & mw[3]) != ~0u;
-        if (part) apply_mask128(s, mw);
-      } else {
+      // (NA: keys outside the row's window already carry the penalty from the S MMA)
+      if constexpr (!NA) {
         if (valid < C::kBN) mask_tail(s, valid);
       }
       // Speculative pass (bf16): exponentiate with the running max m_use and keep the result
@@ -807,9 +869,7 @@ __global__ void __launch_bounds__(384, 1)
       if (slow) {
         if (j > 0 && C::kSpeculative) {
           tmem_ld128_sync(tS, s);
-          if constexpr (NA) {
-            if (part) apply_mask128(s, mw);
-          } else {
+          if constexpr (!NA) {
             if (valid < C::kBN) mask_tail(s, valid);
           }
         }
@@ -823,7 +883,13 @@ __global__ void __launch_bounds__(384, 1)
           exp_pass<FP8, C::kEmuMask>(s, clj, m_use - C::kPShift - lrj, pw, sum);
           sum *= inv_rj;
         } else {
-          const float m_new = fmaxf(m_use, row_max128(s));
+          float rm = row_max128(s);
+          // NA: a row max at the penalty's scale means no key of this tile lies in the row's
+          // window; the row keeps no max (as with -inf keys), so its exponentials stay 0
+          if constexpr (NA) {
+            if (rm < -1.0e27f) rm = -INFINITY;
+          }
+          const float m_new = fmaxf(m_use, rm);
           need = (m_new - m_use) * cl > C::kRescaleLog2;     // true on the first tile
           if (need) {
             alpha = ex2_approx((m_use - m_new) * cl);        // 0 when m_use = -inf
@@ -851,6 +917,25 @@ __global__ void __launch_bounds__(384, 1)
         tmem_st_wait();
       }
       l = fmaf(l, alpha, sum);
+      if constexpr (NA) {
+        // penalty features of this tile's next step, written before P(j) lets the MMA thread
+        // issue that step's S (S(j) is complete, so the block is free): the next brick of this
+        // unit, or the first brick of this tile in the CTA's next unit
+        if (j + 1 < n_own) {
+          int ot, oy, ox;
+          w.kv_origin(j + 1, ot, oy, ox);
+          na_write_pen(sX + t * kNaXBytes, row, wt, wy, wx, p.na_Kt, p.na_Ky, p.na_Kx, ot, oy, ox);
+        } else if (j + 1 == nkv && u + static_cast<int>(gridDim.x) < p.n_units) {
+          const NaTile w2 = na_tile(p, u + gridDim.x, t);
+          if (w2.n() > 0) {
+            int a, b, c, wt2, wy2, wx2, ot, oy, ox;
+            na_row_geo(p, w2, row, a, b, c, wt2, wy2, wx2);
+            w2.kv_origin(0, ot, oy, ox);
+            na_write_pen(sX + t * kNaXBytes, row, wt2, wy2, wx2, p.na_Kt, p.na_Ky, p.na_Kx, ot, oy, ox);
+          }
+        }
+        fence_proxy_async_smem();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_p_full + t);

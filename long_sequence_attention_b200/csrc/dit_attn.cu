@@ -249,7 +249,8 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
   static std::atomic<uint64_t> attr_done{0};
   int rc = check_register_split<D, FP8, NA, PARTS>();
   if (rc != DIT_OK) return rc;
-  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8, NA, PARTS>, C::kSmemBytes, attr_done);
+  constexpr int kSmem = AttnSmem<D, FP8, NA>::kBytes;
+  rc = ensure_smem_attr(attn_fwd_kernel<D, FP8, NA, PARTS>, kSmem, attr_done);
   if (rc != DIT_OK) return rc;
   MapSet<PARTS ? kMaxParts : 1> maps;
   std::memset(&maps, 0, sizeof(maps));
@@ -303,7 +304,7 @@ int launch_attn(const QKV& in, const AttnParams& prm, cudaStream_t st) {
   const int reserve = g_sm_reserve.load();
   const int slots = sms - reserve > 1 ? sms - reserve : 1;
   const int grid = pr.n_units < slots ? pr.n_units : slots;
-  attn_fwd_kernel<D, FP8, NA, PARTS><<<grid, C::kThreads, C::kSmemBytes, st>>>(maps, pr);
+  attn_fwd_kernel<D, FP8, NA, PARTS><<<grid, C::kThreads, kSmem, st>>>(maps, pr);
   return cudaGetLastError() == cudaSuccess ? DIT_OK : DIT_ERR_CUDA;
 }
 
@@ -521,7 +522,9 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
   if (B < 1 || H < 1 || T < 1 || Y < 1 || X < 1 || B > 65535 || H > 65535) return DIT_ERR_INVALID_ARG;
   if (Kt < 1 || Ky < 1 || Kx < 1 || Kt % 2 == 0 || Ky % 2 == 0 || Kx % 2 == 0 || Kt > T || Ky > Y || Kx > X)
     return DIT_ERR_INVALID_ARG;
-  if (!(scale > 0.0f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
+  // (keys outside a query's window get a score penalty of -2^100, which must dominate
+  // scale * log2(e) times any score difference)
+  if (!(scale >= 1e-20f) || !std::isfinite(scale)) return DIT_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return DIT_ERR_UNSUPPORTED;
   const long long S = static_cast<long long>(T) * Y * X;
   if (S > 0x7FFFFFFFLL || static_cast<long long>(B) * H * S > (1LL << 40)) return DIT_ERR_INVALID_ARG;

@@ -330,6 +330,23 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t smem_addr, uint32_t
   return d;
 }
 
+// Shared-memory matrix descriptor, no swizzle, K-major: core matrices of 8 rows x 16 bytes
+// (rows 16 bytes apart), lbo_bytes between core matrices along K, sbo_bytes between 8-row
+// groups.
+__device__ __forceinline__ uint64_t smem_desc_noswz(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= 1ull << 46;
+  return d;
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy (MMA, TMA).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Instruction descriptor for kind::f16 / kind::f8f6f4 with fp32 accumulation.
 //   ab_format: 1 = bf16 (kind::f16), 0 = e4m3 (kind::f8f6f4)
 //   b_mn_major: B operand stored N-contiguous (true for V in P.V)
