@@ -677,21 +677,6 @@ def run_ours(args, rank, local_rank, world):
     print(json.dumps(line), flush=True)
 
 
-def na3d_tiles(grid, kernel) -> int:
-    """KV tiles the neighborhood kernel visits over all units of one head (its own rule:
-    units of two 4x4x8 bricks stacked along y; the union of their windows covered by bricks
-    laid from the union's origin)."""
-    def ws(i, K, L):
-        return min(max(i - K // 2, 0), L - K)
-
-    def span(a, ext, K, L, b):
-        last = min(a + ext, L) - 1
-        return (ws(last, K, L) + K - ws(a, K, L) + b - 1) // b
-    T, Y, X = grid
-    return sum(span(t, 4, kernel[0], T, 4) * span(y, 8, kernel[1], Y, 4) * span(x, 8, kernel[2], X, 8)
-               for t in range(0, T, 4) for y in range(0, Y, 8) for x in range(0, X, 8))
-
-
 def run_na3d_context(lsa, dev, stream, ranks, reps: int = 10):
     """3-D neighborhood attention on the video token grid (21 x 30 x 52, 40 heads, D = 128,
     7 x 7 x 7 window), reported beside the step: its own kernel time, useful FLOP/s (keys in
@@ -720,12 +705,14 @@ def run_na3d_context(lsa, dev, stream, ranks, reps: int = 10):
     stream.synchronize()
     ms = ranks.max(t0.elapsed_time(t1)) / reps
     useful = 4.0 * H * S * kernel[0] * kernel[1] * kernel[2] * D
-    executed = 4.0 * H * na3d_tiles(grid, kernel) * 256 * 128 * D
+    plan = lsa.dit_na3d_plan(*grid, *kernel)           # the kernel's own tiling (host call)
+    executed = 4.0 * H * plan["steps_per_head"] * 256 * 128 * D
     del q, k, v, out, lse
     return {"grid": list(grid), "window": list(kernel), "heads": H, "D": D, "ms": round(ms, 4),
             "useful_tflops": round(useful * ranks.world / (ms * 1e-3) / 1e12, 2),
             "executed_tflops": round(executed * ranks.world / (ms * 1e-3) / 1e12, 2),
-            "tile_efficiency": round(useful / executed, 4), "call": "dit_na3d_fwd"}
+            "tile_efficiency": round(useful / executed, 4), "q_brick": list(plan["q_brick"]),
+            "steps_per_head": plan["steps_per_head"], "call": "dit_na3d_fwd"}
 
 
 def _time_calls(call, stream, ranks, reps: int = 10) -> float:

@@ -147,6 +147,19 @@ int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* 
                  int T, int Y, int X, int D, int Kt, int Ky, int Kx, float scale, void* stream);
 
 /*
+ * dit_na3d_plan - the tiling dit_na3d_fwd uses for a grid and window (host only, no GPU):
+ * q_brick[0..2] = the Q brick's t, y, x extents (product 128), q_brick[3] = the axis (0 = t,
+ * 1 = y, 2 = x) along which the two Q bricks of a unit lie side by side; *units_per_head =
+ * units of one (b, h); *steps_per_head = KV steps of one (b, h) (each step: one 128-key brick
+ * per Q brick of the unit).  Executed MMA work of a call = 4 * B*H * steps * 256 * 128 * D
+ * FLOPs, plus the window-penalty step (K = 16) of every S tile.
+ *   q_brick int[4], units_per_head, steps_per_head: host pointers, written on success.
+ *   Returns DIT_ERR_INVALID_ARG for the grid / window errors dit_na3d_fwd rejects.
+ */
+int dit_na3d_plan(int T, int Y, int X, int Kt, int Ky, int Kx, int* q_brick, long long* units_per_head,
+                  long long* steps_per_head);
+
+/*
  * dit_attn_fwd_parts - attention whose inputs lie in blocks held by several ranks (possibly on
  * other GPUs, through peer addresses over NVLink), one kernel, no exchange.  The keys are
  * n_kv_parts blocks and the queries n_q_parts blocks of part_rows rows each; block p is held

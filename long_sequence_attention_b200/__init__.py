@@ -57,6 +57,7 @@ def _load() -> ctypes.CDLL:
     lib.dit_attn_fwd_seg.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, vp]
     lib.dit_swap01_chunks.argtypes = [vp, vp, ll, ll, ll, vp]
     lib.dit_na3d_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp]
+    lib.dit_na3d_plan.argtypes = [i, i, i, i, i, i, ctypes.POINTER(i), ctypes.POINTER(ll), ctypes.POINTER(ll)]
     lib.dit_attn_fwd_parts.argtypes = [ctypes.POINTER(vp), i, ctypes.POINTER(vp), ctypes.POINTER(vp), i,
                                        ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, i, i, i, f, vp]
     lib.dit_ipc_export.argtypes = [vp, vp, ctypes.POINTER(ll)]
@@ -190,6 +191,16 @@ def dit_na3d_fwd(q, k, v, out, lse, B: int, H: int, T: int, Y: int, X: int, D: i
                  scale: float, stream=None) -> None:
     _check(lib.dit_na3d_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, T, Y, X, D, Kt, Ky, Kx,
                             float(scale), _stream(stream)), "dit_na3d_fwd")
+
+
+def dit_na3d_plan(T: int, Y: int, X: int, Kt: int, Ky: int, Kx: int):
+    """The neighborhood kernel's tiling for a grid and window (host only): dict with the Q
+    brick (t, y, x), the pairing axis, units and KV steps per head."""
+    qb = (ctypes.c_int * 4)()
+    units, steps = ctypes.c_longlong(0), ctypes.c_longlong(0)
+    _check(lib.dit_na3d_plan(T, Y, X, Kt, Ky, Kx, qb, ctypes.byref(units), ctypes.byref(steps)), "dit_na3d_plan")
+    return {"q_brick": (qb[0], qb[1], qb[2]), "pair_axis": qb[3], "units_per_head": units.value,
+            "steps_per_head": steps.value}
 
 
 def neighborhood_attention(q, k, v, grid, kernel, scale: Optional[float] = None, with_lse: bool = True,

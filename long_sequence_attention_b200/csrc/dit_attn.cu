@@ -131,14 +131,15 @@ long long na_host_count(int a, int ext, int K, int L, int b) {
 }
 
 struct NaChoice {
-  int qb[3];   // Q brick extents (t, y, x)
-  int pax;     // axis of the unit's brick pair
-  int nu[3];   // units along t, y, x
+  int qb[3];          // Q brick extents (t, y, x)
+  int pax;            // axis of the unit's brick pair
+  int nu[3];          // units along t, y, x
+  long long steps;    // KV steps of one head
 };
 
 NaChoice na_choose(const int L[3], const int K[3]) {
   static const int kb[3] = {kNaBt, kNaBy, kNaBx};
-  NaChoice best{{kNaBt, kNaBy, kNaBx}, 1, {0, 0, 0}};
+  NaChoice best{{kNaBt, kNaBy, kNaBx}, 1, {0, 0, 0}, 0};
   long long best_cost = -1;
   for (int lt = 0; lt <= 7; ++lt)
     for (int ly = 0; lt + ly <= 7; ++ly) {
@@ -162,7 +163,7 @@ NaChoice na_choose(const int L[3], const int K[3]) {
         const long long cost = steps + kNaUnitCost * units;
         if (best_cost < 0 || cost < best_cost) {
           best_cost = cost;
-          best = NaChoice{{qb[0], qb[1], qb[2]}, pax, {nu[0], nu[1], nu[2]}};
+          best = NaChoice{{qb[0], qb[1], qb[2]}, pax, {nu[0], nu[1], nu[2]}, steps};
         }
       }
     }
@@ -514,6 +515,21 @@ int dit_attn_fwd_seg(const void* q, const void* k, const void* v, void* out, flo
   if (seg < 1) return DIT_ERR_INVALID_ARG;
   return attn_chunk_impl(q, k, v, out, lse, B, H, S, S, D, 0, S, scale, dtype, out_dtype, descale_qkv, stream,
                          false, BlockScales(), seg);
+}
+
+int dit_na3d_plan(int T, int Y, int X, int Kt, int Ky, int Kx, int* q_brick, long long* units_per_head,
+                  long long* steps_per_head) {
+  if (q_brick == nullptr || units_per_head == nullptr || steps_per_head == nullptr) return DIT_ERR_INVALID_ARG;
+  if (T < 1 || Y < 1 || X < 1 || static_cast<long long>(T) * Y * X > 0x7FFFFFFFLL) return DIT_ERR_INVALID_ARG;
+  if (Kt < 1 || Ky < 1 || Kx < 1 || Kt % 2 == 0 || Ky % 2 == 0 || Kx % 2 == 0 || Kt > T || Ky > Y || Kx > X)
+    return DIT_ERR_INVALID_ARG;
+  const int L[3] = {T, Y, X}, K[3] = {Kt, Ky, Kx};
+  const NaChoice ch = na_choose(L, K);
+  for (int d = 0; d < 3; ++d) q_brick[d] = ch.qb[d];
+  q_brick[3] = ch.pax;
+  *units_per_head = static_cast<long long>(ch.nu[0]) * ch.nu[1] * ch.nu[2];
+  *steps_per_head = ch.steps;
+  return DIT_OK;
 }
 
 int dit_na3d_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H, int T, int Y,

@@ -23,3 +23,12 @@ def cuda_lib():
     __graft_entry__._build_module().build()
     import long_sequence_attention_b200 as lsa
     return lsa
+
+
+@pytest.fixture(scope="session")
+def cuda_lib_host():
+    """The binding for host-only calls (no GPU needed): built in-tree if missing or stale."""
+    import __graft_entry__
+    __graft_entry__._build_module().build()
+    import long_sequence_attention_b200 as lsa
+    return lsa
