@@ -171,6 +171,7 @@ def test_na3d_validation(lib):
     assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 96, 3, 3, 3, 0.1, None) == 2   # D
     assert na(A + 8, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 0.1, None) == 3
     assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 0.0, None) == 1   # scale
+    assert na(A, Bp, Cp, O, L, 1, 2, 3, 4, 5, 64, 3, 3, 3, 1e-21, None) == 1  # scale below the penalty's range
 
 
 def test_parts_validation(lib):
