@@ -77,3 +77,28 @@ def test_na3d_rejects_bad_windows(cuda_lib, kernel):
     with pytest.raises(cuda_lib.DitError) as e:
         cuda_lib.neighborhood_attention(x, x.clone(), x.clone(), (3, 4, 5), kernel, 0.1)
     assert e.value.status == cuda_lib.DIT_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("gain,scale", [(8.0, None), (1.0, 1e-6)])
+def test_na3d_score_extremes(cuda_lib, gain, scale):
+    """Keys outside a window carry a -2^100 score penalty: scores 64x the usual size (inputs x8,
+    exact in bf16) and a tiny softmax scale must still give exactly the windowed softmax."""
+    import torch
+    grid, kernel, D = (6, 9, 17), (3, 7, 3), 128
+    S = int(np.prod(grid))
+    host, dev = [], []
+    for i in range(3):
+        x, bits = normal_bf16((1, 2, S, D), 40 + i)
+        t = to_dev_bf16(bits)
+        if i < 2:
+            t = t * gain
+            x = x * gain
+        host.append(x)
+        dev.append(t.contiguous())
+    scale = (1.0 / np.sqrt(D)) if scale is None else scale
+    out, lse = cuda_lib.neighborhood_attention(*dev, grid, kernel, scale)
+    torch.cuda.synchronize()
+    assert cuda_lib.dit_device_status() == 0
+    ro, rl = onb.neighborhood_attention_3d(*host, grid, kernel, scale)
+    m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
+    assert_bf16_parity(m, ("extremes", gain, scale))
