@@ -14,21 +14,24 @@
 // exponentials of one tile overlap the tensor-core work of the other.  The kernel is
 // persistent: a grid of at most one CTA per SM walks the units u = blockIdx.x + k*gridDim.x
 // (query block fastest, so the CTAs running at the same time share a head's K/V in L2).
-// Barrier phases and ring stages follow a per-CTA running count g of KV tiles (every role
-// adds each unit's tile count, which varies per unit only in the neighborhood form), so the
-// next unit's Q load, its first S MMAs and this unit's epilogue overlap.
+// Barrier phases and ring stages follow a per-CTA running count g of KV steps (every role
+// adds each unit's step count, which varies per unit only in the neighborhood form, where
+// each Q tile also has its own K / V ring slots), so the next unit's Q load, its first S MMAs
+// and this unit's epilogue overlap.
 //
 // Instantiations (template <D, FP8, NA, PARTS>): the dense form (bf16 D = 64 / 128, e4m3
 // D = 128, per-tensor or per-block scales, plain or sequence-segmented layouts, optional
 // running (O, LSE) accumulator); NA, 3-D neighborhood attention, where a tile is a brick of
-// tokens and each Q brick visits only the KV bricks of its own rows' windows, with per-row
-// window masks; PARTS, where the query and key rows lie in blocks held by several ranks
+// tokens, each Q brick visits only the KV bricks of its own rows' windows, and the keys of a
+// brick outside a row's window get a score penalty from one more step of the S MMA; PARTS,
+// where the query and key rows lie in blocks held by several ranks
 // (possibly other GPUs) and every tile is loaded from the block that holds it.
 //
 // Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = one query row = one TMEM lane)
 //   warps 4-7  softmax warpgroup for Q tile 1
-//   warp  8    MMA issuer (one thread issues every tcgen05.mma and commit)
+//   warp  8    MMA issuer (one thread issues every tcgen05.mma and commit; NA: each tile's
+//              next P.V + S in whichever order the two tiles become ready)
 //   warp  9    TMA producer (Q once, then a ring of K stages and a ring of V stages)
 //   warp  10   NA only: TMA producer of Q tile 1's K and V tiles (warp 9 then loads tile 0's)
 //   warps 10-11 otherwise idle (they complete the third warpgroup)
