@@ -102,3 +102,21 @@ def test_na3d_score_extremes(cuda_lib, gain, scale):
     ro, rl = onb.neighborhood_attention_3d(*host, grid, kernel, scale)
     m = metrics(host_f64(out), ro, lse.cpu().numpy().astype(np.float64), rl)
     assert_bf16_parity(m, ("extremes", gain, scale))
+
+
+def test_na3d_video_grid_d64_sampled_rows(cuda_lib):
+    """D = 64 on the full video grid (many units per CTA, each Q tile's two-slot K / V rings
+    wrap many times), 4 heads, sampled rows against the oracle."""
+    import torch
+    grid, kernel, D, H = (21, 30, 52), (7, 7, 7), 64, 4
+    S = int(np.prod(grid))
+    host, dev = _case(1, H, grid, D, seed=77)
+    out, lse = cuda_lib.neighborhood_attention(*dev, grid, kernel, 1.0 / np.sqrt(D))
+    torch.cuda.synchronize()
+    assert cuda_lib.dit_device_status() == 0
+    rows = sorted(set(sample_rows(S, 48, seed=11).tolist()) | {52 * 30 * 20, 52 * 30 - 1})
+    heads = [0, 3]
+    ro, rl = onb.neighborhood_attention_3d(host[0][:, heads], host[1][:, heads], host[2][:, heads], grid, kernel,
+                                           1.0 / np.sqrt(D), rows=rows)
+    m = metrics(host_f64(out[:, heads][:, :, rows]), ro, lse[:, heads][:, :, rows].cpu().numpy().astype(np.float64), rl)
+    assert_bf16_parity(m, "video na3d D=64")
